@@ -1,0 +1,92 @@
+"""The growing KV cache after an append, and the ABI's descriptor words.
+
+Test infrastructure (see the package docstring).
+
+After a segment is generated its keys and values join a permanent cache that
+every later segment attends to ([gpts24] "One World, Generated Segment by
+Segment"). Its action tails stay in the cache but are never visible to a
+later segment ([picx] "Action-Aware Causal Attention (Figure 6b)"), so the
+appended tail keys are marked dead.
+
+Cache layout (the library's documented format): K and V are head-major
+``[heads, capacity, 128]``; the descriptor array holds one 32-bit word per
+key:
+
+    bits  0..15  segment index (cache order)
+    bit  16      token is an action tail
+    bit  17      alive: visible to later segments (video and head)
+    bit  18      token is in the descriptive head
+    bits 24..29  action index of a tail token (0 otherwise)
+
+Query descriptors are two words per query:
+
+    word 0: bits 0..15 segment index, bit 16 sees earlier segments,
+            bit 17 valid query
+    word 1: bit a set when the query sees tail a of its own segment
+"""
+from __future__ import annotations
+
+from typing import Tuple
+
+import numpy as np
+
+from .rule import FULL_SEGMENT, TAIL, VIDEO, Layout
+
+SEG_MASK = 0xFFFF
+IS_TAIL = 1 << 16
+ALIVE = 1 << 17
+IS_HEAD = 1 << 18
+ACTION_SHIFT = 24
+Q_SEES_PAST = 1 << 16
+Q_VALID = 1 << 17
+
+
+def segment_key_descriptors(segment, segment_index: int) -> np.ndarray:
+    """Descriptor word of each key of one segment, in token order."""
+    words = []
+    nv = segment.num_frames * segment.tokens_per_frame
+    words += [segment_index | ALIVE] * nv                        # video
+    words += [segment_index | ALIVE | IS_HEAD] * segment.head_len  # head
+    for a, act in enumerate(segment.actions):                    # tails: dead later
+        words += [segment_index | IS_TAIL | (a << ACTION_SHIFT)] * act.length
+    return np.asarray(words, dtype=np.uint32)
+
+
+def key_descriptors(segments, first_index: int = 0) -> np.ndarray:
+    parts = [segment_key_descriptors(s, first_index + i) for i, s in enumerate(segments)]
+    return np.concatenate(parts) if parts else np.zeros(0, np.uint32)
+
+
+def query_descriptors(layout: Layout) -> np.ndarray:
+    """[n_queries, 2] words describing what each query sees."""
+    out = np.zeros((layout.n_queries, 2), dtype=np.uint32)
+    for run in layout.runs:
+        sees_past = run.kind == VIDEO or layout.policy == FULL_SEGMENT
+        w0 = run.segment | Q_VALID | (Q_SEES_PAST if sees_past else 0)
+        sp = layout.spans[run.segment]
+        bits = 0
+        for a, (b, e) in enumerate(sp.windows):
+            if run.kind == VIDEO:
+                seen = b <= run.frame < e
+            else:
+                seen = layout.policy == FULL_SEGMENT or (run.kind == TAIL and run.action == a)
+            if seen:
+                bits |= 1 << a
+        out[run.start:run.stop, 0] = w0
+        out[run.start:run.stop, 1] = bits
+    return out
+
+
+def append(cache_k: np.ndarray, cache_v: np.ndarray, cache_desc: np.ndarray,
+           length: int, segment_index: int, segment, k: np.ndarray, v: np.ndarray
+           ) -> Tuple[np.ndarray, np.ndarray, np.ndarray, int]:
+    """Copy a segment's token-major K/V [n, H, d] into the head-major cache
+    at rows [length, length+n) and write its descriptor words."""
+    n = k.shape[0]
+    ck, cv, cd = cache_k.copy(), cache_v.copy(), cache_desc.copy()
+    if length + n > ck.shape[1]:
+        raise ValueError("cache capacity exceeded")
+    ck[:, length:length + n, :] = np.transpose(k, (1, 0, 2))
+    cv[:, length:length + n, :] = np.transpose(v, (1, 0, 2))
+    cd[length:length + n] = segment_key_descriptors(segment, segment_index)
+    return ck, cv, cd, length + n
