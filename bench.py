@@ -1,0 +1,425 @@
+"""Benchmark of the action-aware causal attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload 480p-long-session]
+
+One step is one pass of the whole hot path over one batch: build the mask
+metadata (per-token descriptors, tile schedule, unmasked-pair count) on the
+host and upload it, run the attention forward of the current segment over the
+cache, and append the segment's K/V to the cache (the cache is rolled back to
+its prior segments afterwards so every step sees the same session length).
+
+Metric: effective attention TFLOP/s counting unmasked work only,
+4 * 128 * heads * A per call, A the unmasked query-key pairs per head (Eq. 6 of
+the Hy-Nomas report). Rank 0 prints one JSON line. With N > 1 (torchrun) each
+rank runs an independent replica of the workload (no data-path collective:
+the path has no exchange step) and `value` is the sum over ranks divided by
+the slowest rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from segment_causal_masked_b200 import workloads as W  # noqa: E402
+
+METRIC = "effective attention TFLOP/s (unmasked work) and % of B200 dense BF16 peak"
+WORKLOADS = {
+    "480p-long-session": W.session_480p_long,
+    "480p-single-turn": W.session_480p_single_turn,
+    "720p-step": W.session_720p,
+}
+KERNEL_SOURCES = ["segment_causal_masked_b200/csrc/sca_kernels.cu",
+                  "segment_causal_masked_b200/csrc/sca_internal.h"]
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def effective_flops(problem, unmasked_pairs: int) -> float:
+    return 4.0 * W.HEAD_DIM * problem.heads * unmasked_pairs
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return dict(json.load(f), source="measured")
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def stored_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel, {}).get(workload)
+    if not e or e.get("kernel_hash") != kernel_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle (baseline and the reference arm only)
+# ---------------------------------------------------------------------------
+
+class OracleSample:
+    """The oracle on `rows` query rows (spread evenly over the query tiles) and
+    `heads` head(s) of the workload, inputs drawn once."""
+
+    def __init__(self, problem, rows: int, heads: int = 1, seed: int = 7):
+        import numpy as np
+        import torch
+
+        from oracle import rule as orule
+
+        torch.set_num_threads(os.cpu_count() or 1)
+        self.p = problem
+        self.lay = orule.Layout.of(problem)
+        nq, nk = problem.n_query_tokens, problem.n_key_tokens
+        self.rows = np.linspace(0, nq - 1, rows).round().astype(np.int64)
+        self.q = W.randn_bf16((nq, heads, W.HEAD_DIM), 1000 * seed).float().numpy()
+        self.k = W.randn_bf16((nk, heads, W.HEAD_DIM), 1000 * seed + 1).float().numpy()
+        self.v = W.randn_bf16((nk, heads, W.HEAD_DIM), 1000 * seed + 2).float().numpy()
+        self.pairs = sum(sum(b - a for a, b in self.lay.ranges(int(r))) for r in self.rows)
+        self.flops = 4.0 * W.HEAD_DIM * heads * self.pairs
+        self.desc = (f"oracle (float64 NumPy) on {rows} query rows x {heads} head(s) of "
+                     f"{problem.name} ({self.pairs} unmasked pairs per head), as effective "
+                     f"TFLOP/s of that sample")
+
+    def run(self) -> float:
+        from oracle import attention as oattn
+
+        t0 = time.perf_counter()
+        oattn.attention_rows(self.lay, self.q, self.k, self.v, self.rows, self.p.softmax_scale)
+        return time.perf_counter() - t0
+
+
+def cpu_threads() -> int:
+    try:
+        import numpy as np  # noqa: F401
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args, problem):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    sample = OracleSample(problem, args.oracle_rows)
+    for _ in range(args.warmup):
+        sample.run()
+    secs = [sample.run() for _ in range(args.steps)]
+    vals = [sample.flops / s / 1e12 for s in secs]
+    desc = sample.desc
+    rows_per_step = args.oracle_rows
+    value = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * statistics.mean(secs), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": problem.name, "queries": problem.n_query_tokens,
+                       "keys": problem.n_key_tokens, "heads": problem.heads,
+                       "head_dim": W.HEAD_DIM, "sample_rows_per_step": rows_per_step},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(),
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the native arm
+# ---------------------------------------------------------------------------
+
+class Session:
+    """One replica of the workload on the current device: a cache holding the
+    prior segments, the current segment's Q/K/V, outputs and metadata."""
+
+    def __init__(self, problem, seed: int):
+        import torch
+
+        from segment_causal_masked_b200 import sca
+
+        self.sca = sca
+        self.p = problem
+        dev = torch.device("cuda", torch.cuda.current_device())
+        h, nc, nq = problem.heads, problem.n_cache_tokens, problem.n_query_tokens
+        self.capacity = nc + nq
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        bf = torch.bfloat16
+        self.k_buf = torch.empty(h, self.capacity, 128, dtype=bf, device=dev)
+        self.v_buf = torch.empty_like(self.k_buf)
+        self.desc = torch.zeros((self.capacity + 127) // 128 * 128, dtype=torch.int32, device=dev)
+        self.cache = sca.KVCache(h, self.capacity, self.k_buf, self.v_buf, self.desc)
+        for seg in problem.cached:
+            k = torch.randn(seg.n_tokens, h, 128, generator=g, device=dev).to(bf)
+            v = torch.randn(seg.n_tokens, h, 128, generator=g, device=dev).to(bf)
+            self.cache.append(seg, k, v)
+        self.n_prior = len(problem.cached)
+        self.q = torch.randn(nq, h, 128, generator=g, device=dev).to(bf)
+        self.k_cur = torch.randn(nq, h, 128, generator=g, device=dev).to(bf)
+        self.v_cur = torch.randn(nq, h, 128, generator=g, device=dev).to(bf)
+        self.o = torch.empty(nq, h, 128, dtype=bf, device=dev)
+        self.lse = torch.empty(h, nq, dtype=torch.float32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.md = sca.Metadata()
+        self.stream = torch.cuda.current_stream()
+        torch.cuda.synchronize()
+
+    def step(self, q=None, k_cur=None, v_cur=None, o=None, ev=None):
+        """One pass of the hot path; `ev` = (start, end) events around the
+        attention kernel."""
+        sca, p = self.sca, self.p
+        s = self.stream.cuda_stream
+        self.md.build(p.cached, p.current, p.textq_policy)
+        self.md.upload(s)
+        if ev is not None:
+            ev[0].record(self.stream)
+        sca.action_causal_attn_fwd(self.cache, self.md, p.heads, self.q if q is None else q,
+                                   self.k_cur if k_cur is None else k_cur,
+                                   self.v_cur if v_cur is None else v_cur,
+                                   self.o if o is None else o, self.lse, p.softmax_scale,
+                                   self.status, s)
+        if ev is not None:
+            ev[1].record(self.stream)
+        self.cache.append(p.current[0], self.k_cur if k_cur is None else k_cur,
+                          self.v_cur if v_cur is None else v_cur, s)
+        self.cache.truncate(self.n_prior)
+
+
+def run_native(args, problem):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}; launch N>1 with torchrun")
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    sess = Session(problem, seed=1000 * 2 + rank)
+    from segment_causal_masked_b200 import sca
+    sca_md = sca.build_segment_mask_metadata(problem.cached, problem.current, problem.textq_policy)
+    counts = sca_md.counts()
+    A = counts["unmasked_pairs"]
+    flops = effective_flops(problem, A)
+
+    # ---- device-resident timing
+    for _ in range(args.warmup):
+        sess.step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start.record(sess.stream)
+    for i in range(args.steps):
+        sess.step(ev=evs[i])
+    t_end.record(sess.stream)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    barrier()
+    if int(sess.status.item()) != 0:
+        raise SystemExit(f"device status {int(sess.status.item())}")
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end))
+    attn_ms = [a.elapsed_time(b) for a, b in evs]
+    attn_avg = max_over_ranks(statistics.mean(attn_ms))
+    ms_step = ms_total / args.steps
+    value = world * flops * args.steps / (ms_total * 1e-3) / 1e12
+
+    # ---- end to end through the API with pinned host buffers
+    nq, h = problem.n_query_tokens, problem.heads
+    pin = dict(pin_memory=True, dtype=torch.bfloat16)
+    hq = sess.q.cpu().pin_memory()
+    hk = sess.k_cur.cpu().pin_memory()
+    hv = sess.v_cur.cpu().pin_memory()
+    ho = torch.empty(nq, h, 128, **pin)
+    dq, dk, dv = torch.empty_like(sess.q), torch.empty_like(sess.k_cur), torch.empty_like(sess.v_cur)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        sess.step(q=dq, k_cur=dk, v_cur=dv)
+        ho.copy_(sess.o, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(sess.stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(sess.stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = world * flops * args.steps / (e2e_ms * 1e-3) / 1e12
+    bytes_in = 3 * hq.numel() * hq.element_size()
+    bytes_out = ho.numel() * ho.element_size()
+
+    if rank == 0:
+        peaks = measured_peaks()
+        peak = float(peaks["bf16_tflops"])
+        achieved = flops / (attn_avg * 1e-3) / 1e12
+        traffic = stored_traffic("attn_fwd_kernel", problem.name)
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": problem.name, "queries": nq, "keys": problem.n_key_tokens,
+                       "cached_segments": len(problem.cached), "heads": h,
+                       "head_dim": W.HEAD_DIM, "unmasked_pairs_per_head": A,
+                       "effective_flop_per_step": flops,
+                       "step": "metadata build+upload, attention forward, kv_cache_append",
+                       "l2": "inputs larger than L2 (cached K/V %.2f GB per tensor)"
+                             % (problem.n_cache_tokens * h * 256 / 1e9),
+                       "parallelism": f"replicas x{world}"},
+            "pct_of_peak": 100.0 * value / world / peak,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "attn_fwd_kernel", "kernel_ms": attn_avg,
+                         "peak_source": f"{peaks['source']} bf16 dense (burst)"},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": bytes_in,
+                    "d2h_bytes_per_step": bytes_out, "ms_per_step": e2e_ms / args.steps},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clock_info,
+        }
+        if not args.no_cpu_baseline:
+            sample = OracleSample(problem, args.baseline_rows)
+            dt = sample.run()
+            line["cpu_baseline"] = {"value": sample.flops / dt / 1e12, "unit": "TFLOP/s",
+                                    "cores": cpu_threads(), "kind": "oracle",
+                                    "sample": sample.desc, "seconds": dt}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="480p-long-session")
+    ap.add_argument("--oracle-rows", type=int, default=384,
+                    help="query rows per step of the reference arm")
+    ap.add_argument("--baseline-rows", type=int, default=1536,
+                    help="query rows of the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
+    problem = WORKLOADS[args.workload]()
+    if args.impl == "reference":
+        return run_reference(args, problem)
+    return run_native(args, problem)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

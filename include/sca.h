@@ -1,0 +1,234 @@
+/*
+ * sca.h - C ABI of libsca: action-aware causal joint attention over a growing
+ * KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * The operation (Hy-Nomas pages):
+ *   - attention is bidirectional inside a segment and causal across segments
+ *     (picx.dev summary, Model Architecture, "Segment-wise Causal Attention");
+ *   - a segment's text is a descriptive head plus action tails a_0..a_n, each
+ *     with a window of latent frames; a query inside an action's window sees
+ *     that tail and the head; heads stay visible to later segments, tails
+ *     never leave their own segment (same page, "Action-Aware Causal
+ *     Attention (Figure 6b)"; onedev.kr review, "무엇과 다른가");
+ *   - after a segment is generated its K/V joins a permanent cache that later
+ *     segments attend to (gpts24.com, "One World, Generated Segment by
+ *     Segment");
+ *   - A, the number of unmasked query-key pairs, is the A_i of Eq. 6 (picx.dev
+ *     summary, Training Infrastructure; xyznot.com, "Dağıtık Paketleme FLOP
+ *     Tahmini").
+ *
+ * Conventions shared by every call:
+ *   - Return value 0 on success, a negative SCA_ERR_* code on failure; the
+ *     calling thread's message is then available from sca_last_error().
+ *     A call that fails validation has no effect (nothing is written, nothing
+ *     is enqueued). No C++ exception crosses this ABI.
+ *   - Device pointers are plain CUDA global-memory addresses owned by the
+ *     caller (e.g. PyTorch tensors). The library owns only its opaque handles.
+ *   - Work is enqueued on the caller's stream (cudaStream_t passed as void*;
+ *     NULL is the legacy default stream) and runs asynchronously; device-side
+ *     failures (a bounded wait that timed out) are reported through the
+ *     optional device status word.
+ *   - Tensors are bf16 with head dimension d = 128. Token-major tensors are
+ *     [tokens][heads][128] contiguous; the cache is head-major
+ *     [heads][capacity][128] contiguous.
+ *   - Every device pointer must be 16-byte aligned (TMA and 16-byte vector
+ *     access); otherwise SCA_ERR_MISALIGNED.
+ */
+#ifndef SCA_H_
+#define SCA_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SCA_API __attribute__((visibility("default")))
+#else
+#define SCA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SCA_HEAD_DIM 128
+#define SCA_TILE 128
+#define SCA_MAX_ACTIONS 32
+#define SCA_MAX_SEGMENTS 65535
+
+enum {
+  SCA_OK = 0,
+  SCA_ERR_INVALID_ARG = -1,   /* bad layout, size or pointer */
+  SCA_ERR_UNSUPPORTED = -2,   /* head_dim != 128, too many segments/tiles */
+  SCA_ERR_MISALIGNED = -3,    /* a device pointer is not 16-byte aligned */
+  SCA_ERR_CAPACITY = -4,      /* the cache cannot hold the appended segment */
+  SCA_ERR_CUDA = -5,          /* a CUDA runtime/driver call failed */
+  SCA_ERR_DEVICE_TIMEOUT = -6,/* a kernel's bounded wait ran out (device status) */
+  SCA_ERR_MISMATCH = -7       /* metadata does not describe this cache */
+};
+
+/* Text-query convention. The pages state what video queries see; for text
+ * queries they are silent.
+ *   SCA_TEXTQ_OWN_TAIL (default): a head query sees its own segment's video
+ *     and head; a query in tail a also sees tail a; no earlier segment.
+ *   SCA_TEXTQ_FULL_SEGMENT: a text query sees its whole own segment and, like
+ *     a video query, the video and heads of earlier segments. */
+enum { SCA_TEXTQ_OWN_TAIL = 0, SCA_TEXTQ_FULL_SEGMENT = 1 };
+
+/* Tile classes of the schedule. */
+enum { SCA_TILE_EMPTY = 0, SCA_TILE_PARTIAL = 1, SCA_TILE_FULL = 2 };
+
+/* Key descriptor word (one per key; the cache's descriptor array and the
+ * current segments' keys):
+ *   bits 0..15 segment index (cache segments first, in time order),
+ *   bit 16 action tail, bit 17 alive (visible to later segments: video and
+ *   head), bit 18 descriptive head, bits 24..29 action index of a tail.
+ * Query descriptor: two words per query,
+ *   word 0: bits 0..15 segment index, bit 16 sees earlier segments,
+ *           bit 17 valid query;
+ *   word 1: bit a set when the query sees tail a of its own segment. */
+#define SCA_DESC_SEG_MASK 0xFFFFu
+#define SCA_DESC_TAIL (1u << 16)
+#define SCA_DESC_ALIVE (1u << 17)
+#define SCA_DESC_HEAD (1u << 18)
+#define SCA_DESC_ACTION_SHIFT 24
+#define SCA_QDESC_SEES_PAST (1u << 16)
+#define SCA_QDESC_VALID (1u << 17)
+
+/* One segment's layout. Token order inside a segment: video frame by frame
+ * (num_frames * tokens_per_frame tokens), then the head (head_len tokens),
+ * then tail 0, tail 1, ... (action_len[a] tokens each). Action a's window is
+ * the half-open latent-frame range [action_begin[a], action_end[a]) local to
+ * the segment. Requirements: num_frames >= 1, tokens_per_frame >= 1,
+ * head_len >= 0, 0 <= num_actions <= 32, action_len[a] >= 1,
+ * 0 <= begin < end <= num_frames. The arrays are read during the call only. */
+typedef struct sca_segment {
+  int32_t num_frames;
+  int32_t tokens_per_frame;
+  int32_t head_len;
+  int32_t num_actions;
+  const int32_t* action_len;
+  const int32_t* action_begin;
+  const int32_t* action_end;
+} sca_segment;
+
+typedef struct sca_metadata sca_metadata; /* mask metadata + tile schedule */
+typedef struct sca_kv_cache sca_kv_cache; /* growing KV cache */
+
+/* ---------------------------------------------------------------------------
+ * Metadata: per-token descriptors and the block-sparse tile schedule.
+ *
+ * Keys are the tokens of `cached` (in time order) followed by those of
+ * `current`; queries are the tokens of `current`. With n_cached = 0 and
+ * several current segments this is a packed training-shaped call.
+ *
+ * Tiles: query tile i = queries [128 i, 128 i + 128). Key tiles are 128
+ * consecutive keys of one source: cache tiles t < nC = ceil(n_cache/128)
+ * cover cache keys [128 t, 128 t + 128); tile nC + u covers current keys
+ * [128 u, 128 u + 128). A (query tile, key tile) pair is FULL when all
+ * 128x128 positions exist and are visible, EMPTY when no existing position is
+ * visible, PARTIAL otherwise. The schedule lists each query tile's non-EMPTY
+ * key tiles in ascending order (CSR).
+ * ------------------------------------------------------------------------- */
+
+/* Create an empty handle. */
+SCA_API int sca_metadata_create(sca_metadata** out);
+
+/* Build descriptors, schedule and A on the host (no GPU needed). Replaces the
+ * handle's previous contents. Requires n_current >= 1 and
+ * n_cached + n_current <= 65535. SCA_ERR_INVALID_ARG on a bad layout. */
+SCA_API int sca_build_segment_mask_metadata(sca_metadata* md,
+                                    const sca_segment* cached, int32_t n_cached,
+                                    const sca_segment* current, int32_t n_current,
+                                    int32_t textq_policy);
+
+/* Sizes and totals of the last build. Any output pointer may be NULL.
+ *   unmasked_pairs: A (pairs whose mask entry is not -inf), per head;
+ *   n_queries / n_cache_keys: token counts; n_q_tiles, n_kv_tiles: tiles;
+ *   nnz / n_full / n_partial: entries of the schedule and their classes. */
+SCA_API int sca_metadata_get_counts(const sca_metadata* md, int64_t* unmasked_pairs,
+                            int64_t* n_queries, int64_t* n_cache_keys,
+                            int32_t* n_q_tiles, int32_t* n_kv_tiles, int64_t* nnz,
+                            int64_t* n_full, int64_t* n_partial);
+
+/* Host views of the schedule (CSR: row_ptr[n_q_tiles+1], kv_tile[nnz],
+ * flag[nnz] with SCA_TILE_PARTIAL/FULL) and of the descriptors of the
+ * current keys (key_desc[n_queries]) and queries (query_desc[2 n_queries]).
+ * The pointers stay valid until the next build or destroy. */
+SCA_API int sca_metadata_get_schedule(const sca_metadata* md, const int32_t** row_ptr,
+                              const int32_t** kv_tile, const uint8_t** flag);
+SCA_API int sca_metadata_get_descriptors(const sca_metadata* md, const uint32_t** key_desc,
+                                 const uint32_t** query_desc);
+
+/* Copy the device-side part (descriptors and the kernel's work list) to the
+ * GPU, on `stream`, through a pinned staging buffer the handle owns. Device
+ * and staging buffers grow on demand (the call that grows them allocates and
+ * may synchronize); a rebuilt handle of the same size reuses them. The
+ * staging buffer is only rewritten after the previous upload has completed. */
+SCA_API int sca_metadata_upload(sca_metadata* md, void* stream);
+
+SCA_API void sca_metadata_destroy(sca_metadata* md);
+
+/* ---------------------------------------------------------------------------
+ * KV cache. The caller allocates, the cache object only records them:
+ *   k_buf, v_buf: bf16 [heads][capacity][128] (head-major);
+ *   desc_buf:     uint32 [round_up(capacity, 128)] key descriptor words.
+ * ------------------------------------------------------------------------- */
+SCA_API int sca_kv_cache_create(sca_kv_cache** out, int32_t heads, int32_t head_dim,
+                        int64_t capacity, void* k_buf, void* v_buf, void* desc_buf);
+
+/* Append one segment: copy its keys and values k, v (bf16 token-major
+ * [n][heads][128], n = the segment's token count) into cache rows
+ * [length, length + n) of every head with 16-byte coalesced stores, write its
+ * key descriptors with the tails marked dead (alive bit clear), and advance
+ * the length. SCA_ERR_CAPACITY if length + n > capacity. */
+SCA_API int sca_kv_cache_append(sca_kv_cache* cache, const sca_segment* segment,
+                        const void* k, const void* v, void* stream);
+
+/* Forget every segment after the first n_segments (host-side; the buffers
+ * keep their bytes). */
+SCA_API int sca_kv_cache_truncate(sca_kv_cache* cache, int32_t n_segments);
+
+/* Length in keys and number of segments. Either pointer may be NULL. */
+SCA_API int sca_kv_cache_get(const sca_kv_cache* cache, int64_t* length, int32_t* n_segments);
+
+SCA_API void sca_kv_cache_destroy(sca_kv_cache* cache);
+
+/* ---------------------------------------------------------------------------
+ * Attention forward.
+ *
+ * For every head h and query i (a token of the metadata's current segments):
+ *   s_ik = softmax_scale * <q_ih, k_kh> for the keys k that i may see,
+ *   o_ih = sum_k softmax_k(s_i) v_kh,  lse[h][i] = log sum_k exp(s_ik),
+ * keys being the cache's keys followed by k_cur. bf16 inputs and outputs,
+ * fp32 accumulation. Arguments:
+ *   cache  : may be NULL when the metadata has no cached segment; otherwise
+ *            its segments must be exactly the metadata's cached layout
+ *            (SCA_ERR_MISMATCH) and its heads the call's heads;
+ *   md     : built and uploaded (sca_metadata_upload) before this call;
+ *   q, k_cur, v_cur, o : bf16 token-major [n_queries][heads][128];
+ *   lse    : fp32 [heads][n_queries] natural-log sum-exp, or NULL;
+ *   dev_status : device int32 (or NULL); left unchanged on success, set to
+ *            SCA_ERR_DEVICE_TIMEOUT if a bounded wait in the kernel ran out;
+ *   stream : the caller's stream.
+ * The call allocates nothing. A query that sees no key gets o = 0 and
+ * lse = -inf. */
+SCA_API int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md,
+                               int32_t heads, const void* q, const void* k_cur,
+                               const void* v_cur, void* o, float* lse,
+                               float softmax_scale, int32_t* dev_status, void* stream);
+
+/* Message of the calling thread's last failure ("" if none). */
+SCA_API const char* sca_last_error(void);
+
+/* ---------------------------------------------------------------------------
+ * Self-test of the device-side bounded wait: one block waits on an mbarrier
+ * that nothing completes, gives up after `timeout_ns` nanoseconds, writes
+ * SCA_ERR_DEVICE_TIMEOUT to *dev_status and returns. Exists so the timeout
+ * path can be exercised without any real hang.
+ * ------------------------------------------------------------------------- */
+SCA_API int sca_debug_bounded_wait(int32_t* dev_status, int64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SCA_H_ */

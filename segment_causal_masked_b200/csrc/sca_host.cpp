@@ -1,0 +1,626 @@
+// Host runtime of libsca: error state, the mask-metadata builder (per-token
+// descriptors, block-sparse tile schedule, unmasked-pair count), the KV-cache
+// object, metadata upload, and argument validation for the kernels.
+//
+// The visibility rule is the action-aware causal attention of the Hy-Nomas
+// pages (picx.dev summary, Model Architecture, "Segment-wise Causal
+// Attention" and "Action-Aware Causal Attention (Figure 6b)"; onedev.kr
+// review, "무엇과 다른가"). Here it is evaluated as a predicate on descriptor
+// words, the same predicate the attention kernel applies on PARTIAL tiles.
+
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <numeric>
+
+#include "sca_internal.h"
+
+namespace sca {
+
+static thread_local std::string g_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_error = buf;
+  return code;
+}
+
+int check_cuda(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return SCA_OK;
+  return fail(SCA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool SegLayout::same(const SegLayout& o) const {
+  if (F != o.F || G != o.G || h != o.h || n_act != o.n_act) return false;
+  for (int a = 0; a < n_act; ++a)
+    if (len[a] != o.len[a] || beg[a] != o.beg[a] || end[a] != o.end[a]) return false;
+  return true;
+}
+
+int read_segment(const sca_segment* s, SegLayout* out) {
+  if (!s) return fail(SCA_ERR_INVALID_ARG, "null segment");
+  if (s->num_frames < 1 || s->tokens_per_frame < 1 || s->head_len < 0)
+    return fail(SCA_ERR_INVALID_ARG,
+                "segment needs num_frames >= 1, tokens_per_frame >= 1, head_len >= 0 "
+                "(got %d, %d, %d)", s->num_frames, s->tokens_per_frame, s->head_len);
+  if (s->num_actions < 0 || s->num_actions > SCA_MAX_ACTIONS)
+    return fail(SCA_ERR_INVALID_ARG, "num_actions must be in [0, %d] (got %d)",
+                SCA_MAX_ACTIONS, s->num_actions);
+  if (s->num_actions > 0 && (!s->action_len || !s->action_begin || !s->action_end))
+    return fail(SCA_ERR_INVALID_ARG, "null action arrays");
+  SegLayout L;
+  L.F = s->num_frames;
+  L.G = s->tokens_per_frame;
+  L.h = s->head_len;
+  L.n_act = s->num_actions;
+  for (int a = 0; a < L.n_act; ++a) {
+    L.len[a] = s->action_len[a];
+    L.beg[a] = s->action_begin[a];
+    L.end[a] = s->action_end[a];
+    if (L.len[a] < 1 || L.beg[a] < 0 || L.beg[a] >= L.end[a] || L.end[a] > L.F)
+      return fail(SCA_ERR_INVALID_ARG,
+                  "action %d needs length >= 1 and 0 <= begin < end <= num_frames "
+                  "(got length %d, window [%d, %d), %d frames)",
+                  a, L.len[a], L.beg[a], L.end[a], L.F);
+  }
+  if (L.n_tokens() > (int64_t(1) << 31) - 1)
+    return fail(SCA_ERR_UNSUPPORTED, "segment has more than 2^31-1 tokens");
+  *out = L;
+  return SCA_OK;
+}
+
+uint32_t key_descriptor(const SegLayout& s, uint32_t seg, int64_t t) {
+  const int64_t nv = s.n_video();
+  if (t < nv) return seg | SCA_DESC_ALIVE;
+  if (t < nv + s.h) return seg | SCA_DESC_ALIVE | SCA_DESC_HEAD;
+  int64_t r = t - nv - s.h;
+  int a = 0;
+  while (a < s.n_act - 1 && r >= s.len[a]) r -= s.len[a++];
+  return seg | SCA_DESC_TAIL | (uint32_t(a) << SCA_DESC_ACTION_SHIFT);
+}
+
+// The pair predicate: may a query described by (q0, q1) see key `k`?
+static inline bool visible(uint32_t q0, uint32_t q1, uint32_t k) {
+  if (!(q0 & SCA_QDESC_VALID)) return false;
+  const uint32_t qs = q0 & SCA_DESC_SEG_MASK, ks = k & SCA_DESC_SEG_MASK;
+  if (ks == qs)  // own segment: everything but the tails outside the query's set
+    return !(k & SCA_DESC_TAIL) || ((q1 >> ((k >> SCA_DESC_ACTION_SHIFT) & 31u)) & 1u);
+  // earlier segment: its live (video, head) keys, if the query looks back
+  return ks < qs && (q0 & SCA_QDESC_SEES_PAST) && (k & SCA_DESC_ALIVE);
+}
+
+namespace {
+
+// What one tile holds, enough to classify a (query tile, key tile) pair.
+struct TileSummary {
+  uint32_t seg_min = 0xFFFFFFFFu, seg_max = 0;
+  bool oob = false;          // fewer than 128 existing rows
+  bool all_flag = true;      // every row sees the past / every key alive
+  bool any_flag = false;
+  std::vector<uint64_t> vals;  // distinct descriptors (query: q0 | q1 << 32)
+  void add(uint64_t v, uint32_t seg, bool flag) {
+    seg_min = std::min(seg_min, seg);
+    seg_max = std::max(seg_max, seg);
+    all_flag &= flag;
+    any_flag |= flag;
+    if (std::find(vals.begin(), vals.end(), v) == vals.end()) vals.push_back(v);
+  }
+};
+
+uint8_t classify(const TileSummary& q, const TileSummary& k) {
+  if (q.vals.empty() || k.vals.empty()) return SCA_TILE_EMPTY;
+  if (k.seg_min > q.seg_max) return SCA_TILE_EMPTY;   // only later segments
+  if (k.seg_max < q.seg_min) {                          // only earlier segments
+    if (!q.any_flag || !k.any_flag) return SCA_TILE_EMPTY;
+    if (q.all_flag && k.all_flag && !q.oob && !k.oob) return SCA_TILE_FULL;
+    return SCA_TILE_PARTIAL;
+  }
+  bool any = false, all = !q.oob && !k.oob;
+  for (uint64_t qv : q.vals)
+    for (uint64_t kv : k.vals) {
+      const bool v = visible(uint32_t(qv), uint32_t(qv >> 32), uint32_t(kv));
+      any |= v;
+      all &= v;
+    }
+  return !any ? SCA_TILE_EMPTY : (all ? SCA_TILE_FULL : SCA_TILE_PARTIAL);
+}
+
+}  // namespace
+
+}  // namespace sca
+
+using namespace sca;
+
+extern "C" {
+
+const char* sca_last_error(void) { return g_error.c_str(); }
+
+int sca_metadata_create(sca_metadata** out) {
+  if (!out) return fail(SCA_ERR_INVALID_ARG, "null output pointer");
+  *out = new (std::nothrow) sca_metadata();
+  return *out ? SCA_OK : fail(SCA_ERR_INVALID_ARG, "out of host memory");
+}
+
+void sca_metadata_destroy(sca_metadata* md) {
+  if (!md) return;
+  if (md->upload_done) {
+    cudaEventSynchronize(md->upload_done);
+    cudaEventDestroy(md->upload_done);
+  }
+  if (md->dev) cudaFree(md->dev);
+  if (md->pinned) cudaFreeHost(md->pinned);
+  delete md;
+}
+
+int sca_build_segment_mask_metadata(sca_metadata* md, const sca_segment* cached,
+                                    int32_t n_cached, const sca_segment* current,
+                                    int32_t n_current, int32_t policy) {
+  if (!md) return fail(SCA_ERR_INVALID_ARG, "null metadata handle");
+  if (n_cached < 0 || n_current < 1)
+    return fail(SCA_ERR_INVALID_ARG, "need n_cached >= 0 and n_current >= 1");
+  if (int64_t(n_cached) + n_current > SCA_MAX_SEGMENTS)
+    return fail(SCA_ERR_UNSUPPORTED, "more than %d segments", SCA_MAX_SEGMENTS);
+  if ((n_cached > 0 && !cached) || !current)
+    return fail(SCA_ERR_INVALID_ARG, "null segment array");
+  if (policy != SCA_TEXTQ_OWN_TAIL && policy != SCA_TEXTQ_FULL_SEGMENT)
+    return fail(SCA_ERR_INVALID_ARG, "unknown text-query policy %d", policy);
+
+  std::vector<SegLayout> segs((size_t)n_cached + n_current);
+  for (int i = 0; i < n_cached; ++i) {
+    int rc = read_segment(&cached[i], &segs[i]);
+    if (rc) return rc;
+  }
+  for (int j = 0; j < n_current; ++j) {
+    int rc = read_segment(&current[j], &segs[size_t(n_cached) + j]);
+    if (rc) return rc;
+  }
+  int64_t n_cache = 0, n_q = 0;
+  for (int i = 0; i < n_cached; ++i) n_cache += segs[i].n_tokens();
+  for (int j = 0; j < n_current; ++j) n_q += segs[size_t(n_cached) + j].n_tokens();
+  if (n_cache > (int64_t(1) << 31) - 1 || n_q > (int64_t(1) << 31) - 256)
+    return fail(SCA_ERR_UNSUPPORTED, "more than 2^31 keys or queries");
+  const int64_t n_ct = (n_cache + SCA_TILE - 1) / SCA_TILE;
+  const int64_t n_ut = (n_q + SCA_TILE - 1) / SCA_TILE;
+  if (n_ct + n_ut > int64_t(kPairTileMask))
+    return fail(SCA_ERR_UNSUPPORTED, "more than 2^24 key tiles");
+
+  // --- descriptors ---------------------------------------------------------
+  std::vector<uint32_t> kdesc_cache((size_t)n_cache);
+  {
+    int64_t pos = 0;
+    for (int i = 0; i < n_cached; ++i)
+      for (int64_t t = 0; t < segs[i].n_tokens(); ++t)
+        kdesc_cache[size_t(pos++)] = key_descriptor(segs[i], uint32_t(i), t);
+  }
+  std::vector<uint32_t> kdesc_cur((size_t)n_q), qdesc((size_t)(2 * n_q));
+  int64_t A = 0;
+  {
+    // alive keys of all earlier segments, for A
+    std::vector<int64_t> alive_before(segs.size() + 1, 0);
+    for (size_t s = 0; s < segs.size(); ++s)
+      alive_before[s + 1] = alive_before[s] + segs[s].n_video() + segs[s].h;
+    const bool full = policy == SCA_TEXTQ_FULL_SEGMENT;
+    int64_t q = 0;
+    for (int j = 0; j < n_current; ++j) {
+      const uint32_t g = uint32_t(n_cached + j);
+      const SegLayout& S = segs[g];
+      const int64_t own_live = S.n_video() + S.h;
+      auto emit = [&](int64_t count, uint32_t w0, uint32_t w1) {
+        int64_t seen = own_live + ((w0 & SCA_QDESC_SEES_PAST) ? alive_before[g] : 0);
+        for (int a = 0; a < S.n_act; ++a)
+          if ((w1 >> a) & 1u) seen += S.len[a];
+        A += count * seen;
+        for (int64_t i = 0; i < count; ++i, ++q) {
+          qdesc[size_t(2 * q)] = w0;
+          qdesc[size_t(2 * q + 1)] = w1;
+        }
+      };
+      const uint32_t base = g | SCA_QDESC_VALID;
+      for (int f = 0; f < S.F; ++f) emit(S.G, base | SCA_QDESC_SEES_PAST, S.frame_mask(f));
+      const uint32_t text0 = base | (full ? SCA_QDESC_SEES_PAST : 0u);
+      emit(S.h, text0, full ? S.all_actions() : 0u);
+      for (int a = 0; a < S.n_act; ++a) emit(S.len[a], text0, full ? S.all_actions() : (1u << a));
+    }
+    int64_t pos = 0;
+    for (int j = 0; j < n_current; ++j) {
+      const uint32_t g = uint32_t(n_cached + j);
+      for (int64_t t = 0; t < segs[g].n_tokens(); ++t)
+        kdesc_cur[size_t(pos++)] = key_descriptor(segs[g], g, t);
+    }
+  }
+
+  // --- tile summaries ------------------------------------------------------
+  const int n_qt = int((n_q + SCA_TILE - 1) / SCA_TILE);
+  std::vector<TileSummary> qs((size_t)n_qt), ks((size_t)(n_ct + n_ut));
+  for (int64_t i = 0; i < n_q; ++i) {
+    const uint32_t w0 = qdesc[size_t(2 * i)], w1 = qdesc[size_t(2 * i + 1)];
+    qs[size_t(i / SCA_TILE)].add(uint64_t(w0) | (uint64_t(w1) << 32), w0 & SCA_DESC_SEG_MASK,
+                                 (w0 & SCA_QDESC_SEES_PAST) != 0);
+  }
+  qs[size_t(n_qt - 1)].oob = (n_q % SCA_TILE) != 0;
+  auto add_keys = [&](const std::vector<uint32_t>& d, int64_t n, int64_t tile0) {
+    for (int64_t i = 0; i < n; ++i)
+      ks[size_t(tile0 + i / SCA_TILE)].add(d[size_t(i)], d[size_t(i)] & SCA_DESC_SEG_MASK,
+                                           (d[size_t(i)] & SCA_DESC_ALIVE) != 0);
+    if (n % SCA_TILE) ks[size_t(tile0 + n / SCA_TILE)].oob = true;
+  };
+  add_keys(kdesc_cache, n_cache, 0);
+  add_keys(kdesc_cur, n_q, n_ct);
+
+  // --- classification and CSR ---------------------------------------------
+  std::vector<int32_t> row_ptr(size_t(n_qt) + 1, 0), kv_tile;
+  std::vector<uint8_t> flag;
+  int64_t n_full = 0, n_partial = 0;
+  kv_tile.reserve(size_t(n_qt) * 64);
+  flag.reserve(size_t(n_qt) * 64);
+  for (int qt = 0; qt < n_qt; ++qt) {
+    const TileSummary& Q = qs[size_t(qt)];
+    for (int64_t kt = 0; kt < n_ct + n_ut; ++kt) {
+      const TileSummary& K = ks[size_t(kt)];
+      if (kt < n_ct && K.seg_min > Q.seg_max) { kt = n_ct - 1; continue; }  // rest of cache is later
+      if (kt >= n_ct && K.seg_min > Q.seg_max) break;
+      const uint8_t c = classify(Q, K);
+      if (c == SCA_TILE_EMPTY) continue;
+      kv_tile.push_back(int32_t(kt));
+      flag.push_back(c);
+      (c == SCA_TILE_FULL ? n_full : n_partial) += 1;
+    }
+    row_ptr[size_t(qt) + 1] = int32_t(kv_tile.size());
+    if (kv_tile.size() > size_t(INT32_MAX) - 4096)
+      return fail(SCA_ERR_UNSUPPORTED, "schedule larger than 2^31 entries");
+  }
+
+  // --- kernel work list: query-tile pairs, union of their key tiles --------
+  const int n_pairs = (n_qt + 1) / 2;
+  std::vector<int32_t> pair_ptr(size_t(n_pairs) + 1, 0);
+  std::vector<uint32_t> pair_list;
+  pair_list.reserve(kv_tile.size());
+  for (int p = 0; p < n_pairs; ++p) {
+    const int a = 2 * p, b = 2 * p + 1;
+    int32_t ia = row_ptr[size_t(a)], ea = row_ptr[size_t(a) + 1];
+    int32_t ib = b < n_qt ? row_ptr[size_t(b)] : 0, eb = b < n_qt ? row_ptr[size_t(b) + 1] : 0;
+    while (ia < ea || ib < eb) {
+      const int32_t ta = ia < ea ? kv_tile[size_t(ia)] : INT32_MAX;
+      const int32_t tb = ib < eb ? kv_tile[size_t(ib)] : INT32_MAX;
+      const int32_t t = std::min(ta, tb);
+      uint32_t e = uint32_t(t);
+      if (ta == t) e |= uint32_t(flag[size_t(ia++)]) << 24;
+      if (tb == t) e |= uint32_t(flag[size_t(ib++)]) << 26;
+      pair_list.push_back(e);
+    }
+    pair_ptr[size_t(p) + 1] = int32_t(pair_list.size());
+  }
+  std::vector<int32_t> order((size_t)n_pairs);
+  std::iota(order.begin(), order.end(), 0);
+  std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
+    return pair_ptr[size_t(x) + 1] - pair_ptr[size_t(x)] > pair_ptr[size_t(y) + 1] - pair_ptr[size_t(y)];
+  });
+
+  md->built = true;
+  md->uploaded = false;
+  md->n_cached = n_cached;
+  md->n_current = n_current;
+  md->policy = policy;
+  md->segs.swap(segs);
+  md->n_cache = n_cache;
+  md->n_q = n_q;
+  md->unmasked_pairs = A;
+  md->n_q_tiles = n_qt;
+  md->n_cache_tiles = int32_t(n_ct);
+  md->n_kv_tiles = int32_t(n_ct + n_ut);
+  md->n_pairs = n_pairs;
+  md->n_full = n_full;
+  md->n_partial = n_partial;
+  md->key_desc_cur.swap(kdesc_cur);
+  md->query_desc.swap(qdesc);
+  md->row_ptr.swap(row_ptr);
+  md->kv_tile.swap(kv_tile);
+  md->flag.swap(flag);
+  md->pair_ptr.swap(pair_ptr);
+  md->pair_list.swap(pair_list);
+  md->item_order.swap(order);
+  return SCA_OK;
+}
+
+int sca_metadata_get_counts(const sca_metadata* md, int64_t* unmasked_pairs, int64_t* n_queries,
+                            int64_t* n_cache_keys, int32_t* n_q_tiles, int32_t* n_kv_tiles,
+                            int64_t* nnz, int64_t* n_full, int64_t* n_partial) {
+  if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
+  if (unmasked_pairs) *unmasked_pairs = md->unmasked_pairs;
+  if (n_queries) *n_queries = md->n_q;
+  if (n_cache_keys) *n_cache_keys = md->n_cache;
+  if (n_q_tiles) *n_q_tiles = md->n_q_tiles;
+  if (n_kv_tiles) *n_kv_tiles = md->n_kv_tiles;
+  if (nnz) *nnz = int64_t(md->kv_tile.size());
+  if (n_full) *n_full = md->n_full;
+  if (n_partial) *n_partial = md->n_partial;
+  return SCA_OK;
+}
+
+int sca_metadata_get_schedule(const sca_metadata* md, const int32_t** row_ptr,
+                              const int32_t** kv_tile, const uint8_t** flag) {
+  if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
+  if (row_ptr) *row_ptr = md->row_ptr.data();
+  if (kv_tile) *kv_tile = md->kv_tile.data();
+  if (flag) *flag = md->flag.data();
+  return SCA_OK;
+}
+
+int sca_metadata_get_descriptors(const sca_metadata* md, const uint32_t** key_desc,
+                                 const uint32_t** query_desc) {
+  if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
+  if (key_desc) *key_desc = md->key_desc_cur.data();
+  if (query_desc) *query_desc = md->query_desc.data();
+  return SCA_OK;
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int sca_metadata_upload(sca_metadata* md, void* stream) {
+  if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  if (int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
+  // layout of the device block
+  const size_t nq_pad = size_t(md->n_pairs) * 2 * SCA_TILE;
+  const size_t nk_pad = align_up(size_t(md->n_q), SCA_TILE);
+  size_t off = 0;
+  const size_t off_q = off;     off = align_up(off + nq_pad * 8, 256);
+  const size_t off_k = off;     off = align_up(off + nk_pad * 4, 256);
+  const size_t off_o = off;     off = align_up(off + size_t(md->n_pairs) * 4, 256);
+  const size_t off_p = off;     off = align_up(off + (size_t(md->n_pairs) + 1) * 4, 256);
+  const size_t off_l = off;     off = align_up(off + std::max<size_t>(md->pair_list.size(), 1) * 4, 256);
+  const size_t bytes = off;
+
+  if (md->upload_done) {  // the staging buffer may still feed the previous copy
+    if (int rc = check_cuda(cudaEventSynchronize(md->upload_done), "cudaEventSynchronize")) return rc;
+  } else if (int rc = check_cuda(cudaEventCreateWithFlags(&md->upload_done, cudaEventDisableTiming),
+                                 "cudaEventCreate")) {
+    return rc;
+  }
+  if (md->dev && (md->device != dev || md->dev_bytes < bytes)) {
+    cudaFree(md->dev);
+    md->dev = nullptr;
+    md->dev_bytes = 0;
+  }
+  if (!md->dev) {
+    if (int rc = check_cuda(cudaMalloc(&md->dev, bytes), "cudaMalloc(metadata)")) return rc;
+    md->dev_bytes = bytes;
+    md->device = dev;
+  }
+  if (md->pinned_bytes < bytes) {
+    if (md->pinned) cudaFreeHost(md->pinned);
+    md->pinned = nullptr;
+    md->pinned_bytes = 0;
+    if (int rc = check_cuda(cudaMallocHost(&md->pinned, bytes), "cudaMallocHost(metadata)")) return rc;
+    md->pinned_bytes = bytes;
+  }
+  uint8_t* h = static_cast<uint8_t*>(md->pinned);
+  memset(h, 0, bytes);
+  memcpy(h + off_q, md->query_desc.data(), md->query_desc.size() * 4);  // padding: invalid queries
+  uint32_t* kd = reinterpret_cast<uint32_t*>(h + off_k);
+  memcpy(kd, md->key_desc_cur.data(), md->key_desc_cur.size() * 4);
+  for (size_t i = md->key_desc_cur.size(); i < nk_pad; ++i) kd[i] = SCA_DESC_SEG_MASK;  // never visible
+  memcpy(h + off_o, md->item_order.data(), md->item_order.size() * 4);
+  memcpy(h + off_p, md->pair_ptr.data(), md->pair_ptr.size() * 4);
+  memcpy(h + off_l, md->pair_list.data(), md->pair_list.size() * 4);
+  if (int rc = check_cuda(cudaMemcpyAsync(md->dev, h, bytes, cudaMemcpyHostToDevice, st),
+                          "cudaMemcpyAsync(metadata)"))
+    return rc;
+  if (int rc = check_cuda(cudaEventRecord(md->upload_done, st), "cudaEventRecord")) return rc;
+  md->off_qdesc = off_q;
+  md->off_kdesc = off_k;
+  md->off_order = off_o;
+  md->off_ptr = off_p;
+  md->off_list = off_l;
+  md->uploaded = true;
+  return SCA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// KV cache
+// ---------------------------------------------------------------------------
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int sca_kv_cache_create(sca_kv_cache** out, int32_t heads, int32_t head_dim, int64_t capacity,
+                        void* k_buf, void* v_buf, void* desc_buf) {
+  if (!out) return fail(SCA_ERR_INVALID_ARG, "null output pointer");
+  *out = nullptr;
+  if (head_dim != SCA_HEAD_DIM) return fail(SCA_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (heads < 1 || capacity < 1 || capacity > (int64_t(1) << 31) - 1)
+    return fail(SCA_ERR_INVALID_ARG, "need heads >= 1 and 1 <= capacity < 2^31");
+  if (!k_buf || !v_buf || !desc_buf) return fail(SCA_ERR_INVALID_ARG, "null cache buffer");
+  if (!aligned16(k_buf) || !aligned16(v_buf) || !aligned16(desc_buf))
+    return fail(SCA_ERR_MISALIGNED, "cache buffers must be 16-byte aligned");
+  sca_kv_cache* c = new (std::nothrow) sca_kv_cache();
+  if (!c) return fail(SCA_ERR_INVALID_ARG, "out of host memory");
+  c->heads = heads;
+  c->capacity = capacity;
+  c->k = k_buf;
+  c->v = v_buf;
+  c->desc = static_cast<uint32_t*>(desc_buf);
+  *out = c;
+  return SCA_OK;
+}
+
+void sca_kv_cache_destroy(sca_kv_cache* c) { delete c; }
+
+int sca_kv_cache_get(const sca_kv_cache* c, int64_t* length, int32_t* n_segments) {
+  if (!c) return fail(SCA_ERR_INVALID_ARG, "null cache");
+  if (length) *length = c->length;
+  if (n_segments) *n_segments = int32_t(c->segs.size());
+  return SCA_OK;
+}
+
+int sca_kv_cache_truncate(sca_kv_cache* c, int32_t n_segments) {
+  if (!c) return fail(SCA_ERR_INVALID_ARG, "null cache");
+  if (n_segments < 0 || size_t(n_segments) > c->segs.size())
+    return fail(SCA_ERR_INVALID_ARG, "cache holds %zu segments, cannot keep %d",
+                c->segs.size(), n_segments);
+  c->length = n_segments == 0 ? 0 : c->seg_start[size_t(n_segments)];
+  c->segs.resize(size_t(n_segments));
+  c->seg_start.resize(size_t(n_segments) + 1);
+  return SCA_OK;
+}
+
+int sca_kv_cache_append(sca_kv_cache* c, const sca_segment* segment, const void* k,
+                        const void* v, void* stream) {
+  if (!c) return fail(SCA_ERR_INVALID_ARG, "null cache");
+  SegLayout L;
+  if (int rc = read_segment(segment, &L)) return rc;
+  if (!k || !v) return fail(SCA_ERR_INVALID_ARG, "null k or v");
+  if (!aligned16(k) || !aligned16(v)) return fail(SCA_ERR_MISALIGNED, "k and v must be 16-byte aligned");
+  if (c->segs.size() >= SCA_MAX_SEGMENTS - 1)
+    return fail(SCA_ERR_UNSUPPORTED, "cache already holds %zu segments", c->segs.size());
+  const int64_t n = L.n_tokens();
+  if (c->length + n > c->capacity)
+    return fail(SCA_ERR_CAPACITY, "cache of capacity %lld holds %lld keys; segment of %lld does not fit",
+                (long long)c->capacity, (long long)c->length, (long long)n);
+  AppendArgs a{};
+  a.k = k;
+  a.v = v;
+  a.k_cache = c->k;
+  a.v_cache = c->v;
+  a.desc = c->desc;
+  a.length = c->length;
+  a.capacity = c->capacity;
+  a.n = int32_t(n);
+  a.heads = c->heads;
+  a.seg_index = uint32_t(c->segs.size());
+  a.n_video = int32_t(L.n_video());
+  a.head_len = L.h;
+  a.n_act = L.n_act;
+  a.tail_start[0] = 0;
+  for (int i = 0; i < L.n_act; ++i) a.tail_start[i + 1] = a.tail_start[i] + L.len[i];
+  if (int rc = check_cuda(launch_append(a, static_cast<cudaStream_t>(stream)), "kv_cache_append launch"))
+    return rc;
+  if (c->seg_start.empty()) c->seg_start.push_back(0);
+  c->segs.push_back(L);
+  c->length += n;
+  c->seg_start.push_back(c->length);
+  return SCA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// attention
+// ---------------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// bf16 tensor of rows of 128 elements, viewed as 3-D (128, dim1, dim2) with the
+// given byte strides of dims 1 and 2; box (64, box1, box2), 128-byte swizzle.
+static int make_map(CUtensorMap* m, const void* base, uint64_t dim1, uint64_t dim2,
+                    uint64_t stride1, uint64_t stride2, uint32_t box1, uint32_t box2) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(SCA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {SCA_HEAD_DIM, dim1, dim2};
+  cuuint64_t strides[2] = {stride1, stride2};
+  cuuint32_t box[3] = {64, box1, box2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SCA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return SCA_OK;
+}
+
+int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md, int32_t heads,
+                               const void* q, const void* k_cur, const void* v_cur, void* o,
+                               float* lse, float softmax_scale, int32_t* dev_status,
+                               void* stream) {
+  if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
+  if (!md->uploaded) return fail(SCA_ERR_INVALID_ARG, "metadata not uploaded");
+  if (heads < 1) return fail(SCA_ERR_INVALID_ARG, "heads must be >= 1");
+  if (!q || !k_cur || !v_cur || !o) return fail(SCA_ERR_INVALID_ARG, "null q, k_cur, v_cur or o");
+  if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(o) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return fail(SCA_ERR_MISALIGNED, "q, k_cur, v_cur, o must be 16-byte aligned (lse 4-byte)");
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale))
+    return fail(SCA_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
+  if (md->n_cached > 0) {
+    if (!cache) return fail(SCA_ERR_MISMATCH, "metadata has cached segments but no cache was given");
+    if (cache->heads != heads) return fail(SCA_ERR_MISMATCH, "cache has %d heads, call has %d", cache->heads, heads);
+    if (cache->segs.size() != size_t(md->n_cached))
+      return fail(SCA_ERR_MISMATCH, "cache holds %zu segments, metadata expects %d",
+                  cache->segs.size(), md->n_cached);
+    for (int i = 0; i < md->n_cached; ++i)
+      if (!cache->segs[size_t(i)].same(md->segs[size_t(i)]))
+        return fail(SCA_ERR_MISMATCH, "cached segment %d differs from the metadata's layout", i);
+  }
+  int dev = 0;
+  if (int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
+  if (dev != md->device) return fail(SCA_ERR_MISMATCH, "metadata was uploaded to another device");
+  if (int64_t(md->n_pairs) * heads > INT32_MAX) return fail(SCA_ERR_UNSUPPORTED, "grid too large");
+
+  const uint64_t row = uint64_t(heads) * SCA_HEAD_DIM * 2;  // bytes per token, token-major
+  AttnMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  int rc = make_map(&maps.q, q, uint64_t(heads), uint64_t(md->n_q), SCA_HEAD_DIM * 2, row, 1, SCA_TILE);
+  if (!rc) rc = make_map(&maps.k_cur, k_cur, uint64_t(heads), uint64_t(md->n_q), SCA_HEAD_DIM * 2, row, 1, SCA_TILE);
+  if (!rc) rc = make_map(&maps.v_cur, v_cur, uint64_t(heads), uint64_t(md->n_q), SCA_HEAD_DIM * 2, row, 1, SCA_TILE);
+  if (!rc && md->n_cache > 0) {
+    const uint64_t hstride = uint64_t(cache->capacity) * SCA_HEAD_DIM * 2;
+    rc = make_map(&maps.k_cache, cache->k, uint64_t(md->n_cache), uint64_t(heads), SCA_HEAD_DIM * 2,
+                  hstride, SCA_TILE, 1);
+    if (!rc) rc = make_map(&maps.v_cache, cache->v, uint64_t(md->n_cache), uint64_t(heads),
+                           SCA_HEAD_DIM * 2, hstride, SCA_TILE, 1);
+  }
+  if (rc) return rc;
+
+  const uint8_t* d = static_cast<const uint8_t*>(md->dev);
+  AttnArgs a{};
+  a.qdesc = reinterpret_cast<const uint2*>(d + md->off_qdesc);
+  a.kdesc_cur = reinterpret_cast<const uint32_t*>(d + md->off_kdesc);
+  a.kdesc_cache = md->n_cache > 0 ? cache->desc : nullptr;
+  a.item_order = reinterpret_cast<const int32_t*>(d + md->off_order);
+  a.pair_ptr = reinterpret_cast<const int32_t*>(d + md->off_ptr);
+  a.pair_list = reinterpret_cast<const uint32_t*>(d + md->off_list);
+  a.o = o;
+  a.lse = lse;
+  a.status = dev_status;
+  a.n_q = int32_t(md->n_q);
+  a.n_cache = int32_t(md->n_cache);
+  a.n_cache_tiles = md->n_cache_tiles;
+  a.heads = heads;
+  a.n_pairs = md->n_pairs;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.timeout_ns = 2000000000ull;
+  return check_cuda(launch_attention(maps, a, static_cast<cudaStream_t>(stream)),
+                    "attention launch");
+}
+
+int sca_debug_bounded_wait(int32_t* dev_status, int64_t timeout_ns, void* stream) {
+  if (!dev_status) return fail(SCA_ERR_INVALID_ARG, "null status");
+  if (timeout_ns < 0 || timeout_ns > 10000000000LL)
+    return fail(SCA_ERR_INVALID_ARG, "timeout must be in [0, 10 s]");
+  return check_cuda(launch_bounded_wait(dev_status, (unsigned long long)timeout_ns,
+                                        static_cast<cudaStream_t>(stream)),
+                    "bounded-wait launch");
+}
+
+}  // extern "C"

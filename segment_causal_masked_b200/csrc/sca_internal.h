@@ -1,0 +1,152 @@
+// Internal declarations shared by the host runtime (sca_host.cpp) and the
+// device kernels (sca_kernels.cu). Not part of the ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "sca.h"
+
+namespace sca {
+
+// Validated copy of one segment's layout.
+struct SegLayout {
+  int32_t F = 0, G = 0, h = 0, n_act = 0;
+  int32_t len[SCA_MAX_ACTIONS] = {};
+  int32_t beg[SCA_MAX_ACTIONS] = {};
+  int32_t end[SCA_MAX_ACTIONS] = {};
+  int64_t n_video() const { return int64_t(F) * G; }
+  int64_t n_tokens() const {
+    int64_t n = n_video() + h;
+    for (int a = 0; a < n_act; ++a) n += len[a];
+    return n;
+  }
+  // bit a set when frame f lies in action a's window
+  uint32_t frame_mask(int f) const {
+    uint32_t m = 0;
+    for (int a = 0; a < n_act; ++a)
+      if (beg[a] <= f && f < end[a]) m |= 1u << a;
+    return m;
+  }
+  uint32_t all_actions() const {
+    return n_act >= 32 ? 0xFFFFFFFFu : ((1u << n_act) - 1u);
+  }
+  bool same(const SegLayout& o) const;
+};
+
+// Sets the thread's message and returns `code`.
+int fail(int code, const char* fmt, ...);
+int check_cuda(cudaError_t e, const char* what);
+int read_segment(const sca_segment* s, SegLayout* out);
+
+// Descriptor word of token `t` (0-based inside the segment).
+uint32_t key_descriptor(const SegLayout& s, uint32_t seg_index, int64_t t);
+
+// ---------------------------------------------------------------------------
+// device-side views
+// ---------------------------------------------------------------------------
+
+// Pair work list entry: bits 0..23 key tile, bits 24..25 class for the
+// first query tile of the pair, bits 26..27 for the second.
+constexpr uint32_t kPairTileMask = 0xFFFFFFu;
+
+struct AttnArgs {
+  // metadata (device)
+  const uint2* qdesc;          // [n_pairs * 256]
+  const uint32_t* kdesc_cur;   // [round_up(n_q, 128)]
+  const uint32_t* kdesc_cache; // [round_up(capacity, 128)] or null
+  const int32_t* item_order;   // [n_pairs] longest list first
+  const int32_t* pair_ptr;     // [n_pairs + 1]
+  const uint32_t* pair_list;   // [pair_ptr[n_pairs]]
+  // outputs
+  void* o;                     // bf16 [n_q][heads][128]
+  float* lse;                  // [heads][n_q] or null
+  int32_t* status;             // device status word or null
+  // sizes
+  int32_t n_q;
+  int32_t n_cache;             // cache keys
+  int32_t n_cache_tiles;
+  int32_t heads;
+  int32_t n_pairs;
+  float scale_log2;            // softmax_scale * log2(e)
+  unsigned long long timeout_ns;
+};
+
+struct AttnMaps {
+  CUtensorMap q, k_cur, v_cur, k_cache, v_cache;
+};
+
+cudaError_t launch_attention(const AttnMaps& maps, const AttnArgs& args, cudaStream_t stream);
+
+struct AppendArgs {
+  const void* k;
+  const void* v;
+  void* k_cache;
+  void* v_cache;
+  uint32_t* desc;
+  int64_t length;       // first row written
+  int64_t capacity;
+  int32_t n;            // tokens of the segment
+  int32_t heads;
+  uint32_t seg_index;
+  int32_t n_video;
+  int32_t head_len;
+  int32_t n_act;
+  int32_t tail_start[SCA_MAX_ACTIONS + 1];  // offsets of the tails after the head
+};
+
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
+cudaError_t launch_bounded_wait(int32_t* status, unsigned long long timeout_ns,
+                                cudaStream_t stream);
+
+size_t attention_smem_bytes();
+
+}  // namespace sca
+
+// ---------------------------------------------------------------------------
+// opaque handles
+// ---------------------------------------------------------------------------
+
+struct sca_metadata {
+  bool built = false;
+  int32_t n_cached = 0, n_current = 0, policy = 0;
+  std::vector<sca::SegLayout> segs;   // cached then current
+  int64_t n_cache = 0;                // cached keys
+  int64_t n_q = 0;                    // queries = current keys
+  int64_t unmasked_pairs = 0;
+  int32_t n_q_tiles = 0, n_cache_tiles = 0, n_kv_tiles = 0, n_pairs = 0;
+  int64_t n_full = 0, n_partial = 0;
+  // host outputs
+  std::vector<uint32_t> key_desc_cur;  // [n_q]
+  std::vector<uint32_t> query_desc;    // [2 n_q]
+  std::vector<int32_t> row_ptr;        // [n_q_tiles + 1]
+  std::vector<int32_t> kv_tile;        // [nnz]
+  std::vector<uint8_t> flag;           // [nnz]
+  std::vector<int32_t> pair_ptr;       // [n_pairs + 1]
+  std::vector<uint32_t> pair_list;
+  std::vector<int32_t> item_order;     // [n_pairs]
+  // device copy
+  bool uploaded = false;
+  int device = -1;
+  void* dev = nullptr;
+  size_t dev_bytes = 0;
+  void* pinned = nullptr;
+  size_t pinned_bytes = 0;
+  cudaEvent_t upload_done = nullptr;
+  size_t off_qdesc = 0, off_kdesc = 0, off_order = 0, off_ptr = 0, off_list = 0;
+};
+
+struct sca_kv_cache {
+  int32_t heads = 0;
+  int64_t capacity = 0;
+  void* k = nullptr;
+  void* v = nullptr;
+  uint32_t* desc = nullptr;
+  int64_t length = 0;
+  std::vector<sca::SegLayout> segs;
+  std::vector<int64_t> seg_start;
+};

@@ -1,0 +1,637 @@
+// Device kernels of libsca for NVIDIA B200 (sm_100a):
+//
+//  * kv_append_kernel   - appends a segment's K/V to the head-major bf16 cache
+//                         with 16-byte coalesced loads and stores and writes its
+//                         key descriptors, tails marked dead (gpts24.com, "One
+//                         World, Generated Segment by Segment"; picx.dev
+//                         summary, "Action-Aware Causal Attention (Figure 6b)").
+//  * attn_fwd_kernel    - flash-style forward of action-aware causal attention:
+//                         TMA-staged Q/K/V tiles, tcgen05 MMAs accumulating in
+//                         tensor memory (S = Q K^T and O += P V, P read from
+//                         tensor memory), online softmax in fp32 with the mask
+//                         evaluated from descriptor words on PARTIAL tiles only.
+//  * bounded_wait_kernel - exercises the timeout path of the bounded mbarrier
+//                         wait every pipeline wait here goes through.
+//
+// Attention CTA organisation (one CTA per (query-tile pair, head)):
+//   warps 0-3  softmax of query tile 0 (one thread per row = TMEM lane)
+//   warps 4-7  softmax of query tile 1
+//   warp  8    TMA producer (Q once, then K_j, V_j into a 4-stage ring)
+//   warp  9    TMEM allocator and MMA issuer (one elected thread)
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,384),
+// O1 [384,512); P_t (bf16 pairs) overwrites the first 64 columns of S_t.
+// The MMA warp ping-pongs the two tiles: while softmax works on tile 0's
+// scores the tensor cores run tile 1's P V and next S, and vice versa.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sca_internal.h"
+
+namespace sca {
+
+// ---------------------------------------------------------------------------
+// kv_cache_append
+// ---------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(256) kv_append_kernel(const AppendArgs a) {
+  const uint4* __restrict__ k = static_cast<const uint4*>(a.k);
+  const uint4* __restrict__ v = static_cast<const uint4*>(a.v);
+  uint4* __restrict__ kc = static_cast<uint4*>(a.k_cache);
+  uint4* __restrict__ vc = static_cast<uint4*>(a.v_cache);
+  const int64_t per_tok = int64_t(a.heads) * 16;  // 16-byte chunks per token
+  const int64_t total = int64_t(a.n) * per_tok;
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+    const int64_t tok = i / per_tok;
+    const int32_t rem = int32_t(i - tok * per_tok);
+    const int32_t h = rem >> 4, c = rem & 15;
+    const int64_t dst = ((int64_t(h) * a.capacity) + a.length + tok) * 16 + c;
+    const uint4 kk = __ldg(k + i);
+    const uint4 vv = __ldg(v + i);
+    kc[dst] = kk;
+    vc[dst] = vv;
+  }
+  for (int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; t < a.n; t += stride) {
+    uint32_t d;
+    if (t < a.n_video) {
+      d = a.seg_index | SCA_DESC_ALIVE;
+    } else if (t < int64_t(a.n_video) + a.head_len) {
+      d = a.seg_index | SCA_DESC_ALIVE | SCA_DESC_HEAD;
+    } else {
+      const int32_t r = int32_t(t - a.n_video - a.head_len);
+      int act = 0;
+      while (act + 1 < a.n_act && r >= a.tail_start[act + 1]) ++act;
+      d = a.seg_index | SCA_DESC_TAIL | (uint32_t(act) << SCA_DESC_ACTION_SHIFT);  // dead later
+    }
+    a.desc[a.length + t] = d;
+  }
+}
+
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
+  if (a.n <= 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t chunks = int64_t(a.n) * a.heads * 16;
+  int64_t blocks = (chunks + 255) / 256;
+  blocks = blocks < int64_t(sms) * 8 ? blocks : int64_t(sms) * 8;
+  kv_append_kernel<<<unsigned(blocks), 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Shared control block of one CTA.
+struct Ctl {
+  int32_t abort;   // set by the first wait that times out
+};
+
+// Wait for the phase of `bar` with the given parity. Gives up after
+// `timeout_ns` (or as soon as another thread of the CTA gave up): then sets
+// ctl->abort, writes SCA_ERR_DEVICE_TIMEOUT to *status (if any) and returns
+// false. Every pipeline wait of this file goes through here, so a broken
+// handshake ends the kernel with an error status instead of a hang.
+__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile Ctl* ctl,
+                                          int32_t* status, unsigned long long timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 15u) == 0) {
+      if (ctl->abort) return false;
+      if (global_ns() - t0 > timeout_ns) {
+        ctl->abort = 1;
+        if (status) atomicExch(status, SCA_ERR_DEVICE_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int32_t c0, int32_t c1, int32_t c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version field.
+// K-major (rows of 128 bytes along K, 8-row groups 1024 bytes apart).
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr) {
+  return uint64_t((saddr & 0x3FFFFu) >> 4) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+// MN-major (rows of 128 bytes along N = 64 elements; the next 64 N-elements
+// 16 KB further; 8-row groups along K 1024 bytes apart).
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t saddr) {
+  return uint64_t((saddr & 0x3FFFFu) >> 4) | (uint64_t(16384 >> 4) << 16) |
+         (uint64_t(1024 >> 4) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
+// Instruction descriptor: kind::f16, bf16 A and B, fp32 D, M = 128, N = 128.
+constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) |
+                              ((128u >> 4) << 24);
+constexpr uint32_t kIdescPV = kIdescQK | (1u << 16);  // B (V) is MN-major
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                       uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* r) {
+  uint32_t* u = reinterpret_cast<uint32_t*>(r);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+        "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]),
+        "=r"(u[14]), "=r"(u[15]), "=r"(u[16]), "=r"(u[17]), "=r"(u[18]), "=r"(u[19]),
+        "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]), "=r"(u[25]),
+        "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* r) {
+  const uint32_t* u = reinterpret_cast<const uint32_t*>(r);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+          taddr),
+      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]),
+      "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]),
+      "r"(u[15]), "r"(u[16]), "r"(u[17]), "r"(u[18]), "r"(u[19]), "r"(u[20]), "r"(u[21]),
+      "r"(u[22]), "r"(u[23]), "r"(u[24]), "r"(u[25]), "r"(u[26]), "r"(u[27]), "r"(u[28]),
+      "r"(u[29]), "r"(u[30]), "r"(u[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* u) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]),
+      "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]),
+      "r"(u[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// The pair predicate on descriptor words (layout documented in sca.h).
+__device__ __forceinline__ bool visible(uint32_t q0, uint32_t q1, uint32_t k) {
+  const uint32_t qs = q0 & SCA_DESC_SEG_MASK, ks = k & SCA_DESC_SEG_MASK;
+  const bool own = (ks == qs) && (!(k & SCA_DESC_TAIL) ||
+                                  ((q1 >> ((k >> SCA_DESC_ACTION_SHIFT) & 31u)) & 1u));
+  const bool past = (ks < qs) && (q0 & SCA_QDESC_SEES_PAST) && (k & SCA_DESC_ALIVE);
+  return (q0 & SCA_QDESC_VALID) && (own || past);
+}
+
+// ---------------------------------------------------------------------------
+// attention forward
+// ---------------------------------------------------------------------------
+
+constexpr int kStages = 4;
+constexpr int kThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kHalf = 128 * 64 * 2;  // one 128-row x 64-column bf16 box: 16 KB
+constexpr uint32_t kTile = 2 * kHalf;     // 128 x 128 bf16: 32 KB
+constexpr float kRescaleThreshold = 8.0f; // log2 units: p stays <= 2^8 between rescales
+
+// shared-memory map (offsets from a 1024-aligned base)
+constexpr uint32_t kOffQ = 0;                            // Q0, Q1
+constexpr uint32_t kOffKV = 2 * kTile;                   // ring of K/V tiles
+constexpr uint32_t kOffDesc = kOffKV + kStages * kTile;  // 2 x 128 key descriptors
+constexpr uint32_t kOffBar = kOffDesc + 2 * 128 * 4;
+constexpr uint32_t kBarQ = 0, kBarFull = 1, kBarEmpty = kBarFull + kStages,
+                   kBarS = kBarEmpty + kStages, kBarP = kBarS + 2, kBarO = kBarP + 2,
+                   kBarDrain = kBarO + 2, kNumBars = kBarDrain + 1;
+constexpr uint32_t kOffCtl = kOffBar + kNumBars * 8;
+constexpr uint32_t kOffTmemSlot = kOffCtl + 16;
+constexpr uint32_t kSmemBytes = kOffTmemSlot + 16 + 1024;  // + alignment slack
+
+size_t attention_smem_bytes() { return kSmemBytes; }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_kcur,
+                    const __grid_constant__ CUtensorMap tm_vcur,
+                    const __grid_constant__ CUtensorMap tm_kcache,
+                    const __grid_constant__ CUtensorMap tm_vcache, const AttnArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + kOffBar;
+  auto bar = [&](uint32_t i) { return bar0 + 8 * i; };
+  volatile Ctl* ctl = reinterpret_cast<volatile Ctl*>(smem + kOffCtl);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmemSlot);
+  uint32_t* kdesc_s = reinterpret_cast<uint32_t*>(smem + kOffDesc);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = blockIdx.x / p.heads;
+  const int head = blockIdx.x - rank * p.heads;
+  const int pair = p.item_order[rank];
+  const int list_begin = p.pair_ptr[pair];
+  const int n_iter = p.pair_ptr[pair + 1] - list_begin;
+  const uint32_t* list = p.pair_list + list_begin;
+  const int q_row0 = pair * 256;
+
+  if (threadIdx.x == 0) {
+    ctl->abort = 0;
+    mbar_init(bar(kBarQ), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar(kBarFull + s), 1);
+      mbar_init(bar(kBarEmpty + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(kBarS + t), 1);
+      mbar_init(bar(kBarP + t), 128);
+      mbar_init(bar(kBarO + t), 1);
+    }
+    mbar_init(bar(kBarDrain), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     smem_u32(tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kLoadWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && n_iter > 0) {
+      const uint32_t sQ = sbase + kOffQ;
+      mbar_expect_tx(bar(kBarQ), 2 * kTile);
+      tma_load_3d(sQ, &tm_q, bar(kBarQ), 0, head, q_row0);
+      tma_load_3d(sQ + kHalf, &tm_q, bar(kBarQ), 64, head, q_row0);
+      tma_load_3d(sQ + kTile, &tm_q, bar(kBarQ), 0, head, q_row0 + 128);
+      tma_load_3d(sQ + kTile + kHalf, &tm_q, bar(kBarQ), 64, head, q_row0 + 128);
+      int it = 0;
+      bool ok = true;
+      for (int j = 0; j < n_iter && ok; ++j) {
+        const int tile = int(list[j] & kPairTileMask);
+        for (int kv = 0; kv < 2; ++kv, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = uint32_t(it / kStages) & 1u;
+          if (!wait_bounded(bar(kBarEmpty + s), ph ^ 1u, ctl, p.status, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = sbase + kOffKV + uint32_t(s) * kTile;
+          mbar_expect_tx(bar(kBarFull + s), kTile);
+          if (tile < p.n_cache_tiles) {
+            const CUtensorMap* m = kv ? &tm_vcache : &tm_kcache;
+            tma_load_3d(dst, m, bar(kBarFull + s), 0, tile * 128, head);
+            tma_load_3d(dst + kHalf, m, bar(kBarFull + s), 64, tile * 128, head);
+          } else {
+            const CUtensorMap* m = kv ? &tm_vcur : &tm_kcur;
+            const int row = (tile - p.n_cache_tiles) * 128;
+            tma_load_3d(dst, m, bar(kBarFull + s), 0, head, row);
+            tma_load_3d(dst + kHalf, m, bar(kBarFull + s), 64, head, row);
+          }
+        }
+      }
+      if (!ok) {
+        // drain: let every armed load land before the CTA can exit
+        for (int back = 1; back <= kStages && it - back >= 0; ++back) {
+          const int i2 = it - back;
+          wait_bounded(bar(kBarFull + i2 % kStages), uint32_t(i2 / kStages) & 1u, ctl, nullptr,
+                       p.timeout_ns);
+        }
+        wait_bounded(bar(kBarQ), 0, ctl, nullptr, p.timeout_ns);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_iter > 0) {
+      const uint32_t sQ0 = sbase + kOffQ, sQ1 = sQ0 + kTile;
+      const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
+      auto issue_qk = [&](uint32_t tS, uint32_t sQ, uint32_t sK) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t off = uint32_t(k >> 2) * kHalf + uint32_t(k & 3) * 32;
+          mma_ss(tS, desc_kmajor(sQ + off), desc_kmajor(sK + off), kIdescQK, k > 0);
+        }
+      };
+      auto issue_pv = [&](uint32_t tO, uint32_t tP, uint32_t sV, bool acc) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_ts(tO, tP + uint32_t(k) * 8, desc_mnmajor(sV + uint32_t(k) * 2048), kIdescPV,
+                 (acc || k > 0) ? 1u : 0u);
+      };
+      auto stage_of = [&](int it) { return sbase + kOffKV + uint32_t(it % kStages) * kTile; };
+      auto wait_full = [&](int it) {
+        return wait_bounded(bar(kBarFull + it % kStages), uint32_t(it / kStages) & 1u, ctl,
+                            p.status, p.timeout_ns);
+      };
+      bool ok = wait_bounded(bar(kBarQ), 0, ctl, p.status, p.timeout_ns) && wait_full(0);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(tS0, sQ0, stage_of(0));
+        mma_commit(bar(kBarS + 0));
+        issue_qk(tS1, sQ1, stage_of(0));
+        mma_commit(bar(kBarS + 1));
+        mma_commit(bar(kBarEmpty + 0));
+      }
+      for (int j = 0; j < n_iter && ok; ++j) {
+        const int itV = 2 * j + 1, itK = 2 * j + 2;
+        const uint32_t ph = uint32_t(j) & 1u;
+        const bool more = j + 1 < n_iter;
+        ok = wait_full(itV) && wait_bounded(bar(kBarP + 0), ph, ctl, p.status, p.timeout_ns);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(tO0, tS0, stage_of(itV), j > 0);
+        if (more) {
+          if (!(ok = wait_full(itK))) break;
+          tc_fence_after();
+          issue_qk(tS0, sQ0, stage_of(itK));
+          mma_commit(bar(kBarS + 0));
+        }
+        if (!(ok = wait_bounded(bar(kBarP + 1), ph, ctl, p.status, p.timeout_ns))) break;
+        tc_fence_after();
+        issue_pv(tO1, tS1, stage_of(itV), j > 0);
+        mma_commit(bar(kBarEmpty + itV % kStages));
+        if (more) {
+          issue_qk(tS1, sQ1, stage_of(itK));
+          mma_commit(bar(kBarS + 1));
+          mma_commit(bar(kBarEmpty + itK % kStages));
+        }
+      }
+      mma_commit(bar(kBarO + 0));
+      mma_commit(bar(kBarO + 1));
+      // every MMA has finished before this thread leaves (also on abort)
+      mma_commit(bar(kBarDrain));
+      wait_bounded(bar(kBarDrain), 0, ctl, nullptr, p.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int t = warp >> 2;           // query tile of the pair
+    const int wq = warp & 3;           // TMEM lane quadrant
+    const int r = wq * 32 + lane;      // row in the tile
+    const int q_row = q_row0 + t * 128 + r;
+    const uint2 qd = p.qdesc[q_row];
+    const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
+    const uint32_t tS = lane_base + uint32_t(t) * 128;
+    const uint32_t tO = lane_base + 256 + uint32_t(t) * 128;
+    uint32_t* kds = kdesc_s + t * 128;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_iter; ++j) {
+      const uint32_t e = list[j];
+      const int tile = int(e & kPairTileMask);
+      const uint32_t cls = (e >> (24 + 2 * t)) & 3u;
+      const bool cached = tile < p.n_cache_tiles;
+      const int key0 = (cached ? tile : tile - p.n_cache_tiles) * 128;
+      const int key_limit = (cached ? p.n_cache : p.n_q) - key0;  // existing keys in the tile
+      uint32_t kd = 0;
+      if (cls == SCA_TILE_PARTIAL) kd = cached ? p.kdesc_cache[key0 + r] : p.kdesc_cur[key0 + r];
+      ok = wait_bounded(bar(kBarS + t), uint32_t(j) & 1u, ctl, p.status, p.timeout_ns);
+      if (!__all_sync(0xFFFFFFFFu, ok)) {  // keep the warp's collective TMEM ops uniform
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (cls == SCA_TILE_EMPTY) {
+        // nothing visible for this tile: P = 0
+        uint32_t z[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) z[i] = 0u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_st16(tS + uint32_t(c) * 16, z);
+      } else {
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + uint32_t(c) * 32, s + 32 * c);
+        tmem_wait_ld();
+        if (cls == SCA_TILE_PARTIAL) {
+          kds[r] = kd;
+          named_sync(1 + t, 128);
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            if (c >= key_limit || !visible(qd.x, qd.y, kds[c])) s[c] = -INFINITY;
+          }
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        // The running max only moves when it grows by more than the threshold
+        // (exact: l and O share the stale max until the final division).
+        const float m_cand = mx * p.scale_log2;
+        const bool grow = m_cand > m_run + kRescaleThreshold;
+        const bool rescale = grow && m_run != -INFINITY && j > 0;
+        const float alpha = rescale ? ex2(m_run - m_cand) : 1.f;
+        if (grow) m_run = m_cand;
+        l_run *= alpha;
+        // tcgen05.ld/st are warp-collective: the whole warp rewrites O if any
+        // row needs it (alpha = 1 for the others). O of earlier tiles was
+        // complete when S of this tile completed (in-order MMA pipeline).
+        if (__any_sync(0xFFFFFFFFu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(tO + uint32_t(c) * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(tO + uint32_t(c) * 32, o);
+          }
+        }
+        const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+        float sum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ex2(fmaf(s[32 * c + 2 * i], p.scale_log2, neg_m));
+            const float p1 = ex2(fmaf(s[32 * c + 2 * i + 1], p.scale_log2, neg_m));
+            sum += p0 + p1;
+            pk[i] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tS + uint32_t(c) * 16, pk);
+        }
+        l_run += sum;
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBarP + t));
+    }
+    // ---------------------------------------------------------- epilogue
+    if (ok && n_iter > 0) ok = wait_bounded(bar(kBarO + t), 0, ctl, p.status, p.timeout_ns);
+    if (__all_sync(0xFFFFFFFFu, ok)) {
+      tc_fence_after();
+      const bool store = q_row < p.n_q;
+      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+      uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) +
+                                             (int64_t(q_row) * p.heads + head) * 128);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        if (n_iter > 0) {
+          tmem_ld32(tO + uint32_t(c) * 32, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0.f;
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) w[i] = pack_bf16(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
+        if (store) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            orow[c * 4 + i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+      if (store && p.lse)
+        p.lse[int64_t(head) * p.n_q + q_row] =
+            l_run > 0.f ? (m_run + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+cudaError_t launch_attention(const AttnMaps& maps, const AttnArgs& args, cudaStream_t stream) {
+  static int configured_mask = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 31 && !(configured_mask & (1 << dev))) {
+    e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    configured_mask |= 1 << dev;
+  }
+  const unsigned grid = unsigned(args.n_pairs) * unsigned(args.heads);
+  attn_fwd_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps.q, maps.k_cur, maps.v_cur,
+                                                          maps.k_cache, maps.v_cache, args);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// bounded-wait self-test
+// ---------------------------------------------------------------------------
+
+__global__ void bounded_wait_kernel(int32_t* status, unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t never;
+  __shared__ Ctl ctl;
+  if (threadIdx.x == 0) {
+    ctl.abort = 0;
+    mbar_init(smem_u32(&never), 1);  // nobody ever arrives
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) wait_bounded(smem_u32(&never), 0, &ctl, status, timeout_ns);
+}
+
+cudaError_t launch_bounded_wait(int32_t* status, unsigned long long timeout_ns,
+                                cudaStream_t stream) {
+  bounded_wait_kernel<<<1, 32, 0, stream>>>(status, timeout_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace sca

@@ -1,0 +1,151 @@
+"""Host-side parity of the C++ metadata builder against the oracle (no GPU).
+
+The builder (sca_build_segment_mask_metadata) evaluates a predicate on
+descriptor words; the oracle builds the explicit mask from sets of visible
+key ranges and classifies tiles by brute force. Schedules, descriptors and the
+unmasked-pair count must agree bit for bit.
+"""
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import cache as ocache
+from oracle import rule as orule
+from oracle import schedule as osched
+from segment_causal_masked_b200 import workloads as W
+
+sca = pytest.importorskip("segment_causal_masked_b200.sca")
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _builder(p):
+    return sca.build_segment_mask_metadata(p.cached, p.current, p.textq_policy)
+
+
+def _overlap_problem():
+    segs = (W.Segment(4, 3, 2, (W.Action(2, 0, 3), W.Action(3, 1, 2), W.Action(1, 3, 4))),
+            W.Segment(3, 2, 0, (W.Action(2, 0, 1),)),
+            W.Segment(1, 1, 0))
+    return W.Problem("overlap", (), segs, heads=1)
+
+
+SMALL = [
+    W.tiny_packed(),
+    W.small_session(),
+    W.small_packed(),
+    W.small_packed(seed=21, n_segments=14),
+    W.Problem("small-session-full", W.small_session().cached, W.small_session().current, heads=2,
+              textq_policy=W.TEXTQ_FULL_SEGMENT),
+    _overlap_problem(),
+    W.Problem("one-token", (), (W.Segment(1, 1, 0),), heads=1),
+    W.Problem("no-text-cache", (W.Segment(3, 100, 0),), (W.Segment(2, 70, 5),), heads=1),
+    W.Problem("32-actions", (), (W.Segment(32, 9, 4, tuple(W.Action(3, a, a + 1) for a in range(32))),),
+              heads=1),
+]
+
+
+@pytest.mark.parametrize("p", SMALL, ids=lambda p: p.name)
+def test_schedule_descriptors_and_count_small(p):
+    lay = orule.Layout.of(p)
+    md = _builder(p)
+    c = md.counts()
+    assert c["unmasked_pairs"] == int(lay.mask().sum()) == lay.unmasked_pairs()
+    assert c["n_queries"] == lay.n_queries and c["n_cache_keys"] == lay.n_cache
+    row_ptr, kv, flag = md.schedule()
+    o_row_ptr, o_kv, o_flag = osched.schedule(lay)
+    assert np.array_equal(row_ptr, o_row_ptr)
+    assert np.array_equal(kv, o_kv)
+    assert np.array_equal(flag, o_flag)
+    assert c["n_full"] == int((o_flag == osched.FULL).sum())
+    assert c["n_partial"] == int((o_flag == osched.PARTIAL).sum())
+    kd, qd = md.descriptors()
+    assert np.array_equal(kd, ocache.key_descriptors(p.current, len(p.cached)))
+    assert np.array_equal(qd, ocache.query_descriptors(lay))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("make", [W.session_480p_single_turn, W.session_480p_long, W.session_720p],
+                         ids=["480p-single-turn", "480p-long-session", "720p-step"])
+def test_schedule_full_size(make):
+    p = make()
+    lay = orule.Layout.of(p)
+    md = _builder(p)
+    c = md.counts()
+    assert c["unmasked_pairs"] == lay.unmasked_pairs()
+    row_ptr, kv, flag = md.schedule()
+    o_row_ptr, o_kv, o_flag = osched.schedule(lay)
+    assert np.array_equal(row_ptr, o_row_ptr)
+    assert np.array_equal(kv, o_kv) and np.array_equal(flag, o_flag)
+    kd, qd = md.descriptors()
+    assert np.array_equal(kd, ocache.key_descriptors(p.current, len(p.cached)))
+    assert np.array_equal(qd, ocache.query_descriptors(lay))
+
+
+def test_480p_long_session_totals():
+    """Closed forms: A = 1,923,821,844; 97 query tiles; 1158 + 97 key tiles."""
+    md = _builder(W.session_480p_long())
+    c = md.counts()
+    assert c["unmasked_pairs"] == 1_923_821_844
+    assert c["n_q_tiles"] == 97 and c["n_kv_tiles"] == 1158 + 97
+
+
+@pytest.mark.slow
+def test_packed_360k_sampled_tiles():
+    p = W.packed_360k()
+    lay = orule.Layout.of(p)
+    md = _builder(p)
+    c = md.counts()
+    assert c["unmasked_pairs"] == lay.unmasked_pairs()
+    assert c["n_queries"] == lay.n_queries <= 360_000
+    row_ptr, kv, flag = md.schedule()
+    rng = np.random.default_rng(0)
+    n_qt = c["n_q_tiles"]
+    for qt in sorted({0, n_qt - 1, *rng.choice(n_qt, 6, replace=False).tolist()}):
+        cls = osched.classify_query_tile(lay, qt)
+        nz = np.nonzero(cls)[0]
+        assert np.array_equal(kv[row_ptr[qt]:row_ptr[qt + 1]], nz), qt
+        assert np.array_equal(flag[row_ptr[qt]:row_ptr[qt + 1]], cls[nz]), qt
+
+
+# ---------------------------------------------------------------------------
+# the ABI itself
+# ---------------------------------------------------------------------------
+
+def test_library_exports_every_declared_symbol():
+    with open(os.path.join(ROOT, "include", "sca.h")) as f:
+        declared = set(re.findall(r"SCA_API\s+[\w\s\*]+?\b(sca_\w+)\s*\(", f.read()))
+    assert declared == set(sca.EXPORTED)
+    for name in declared:
+        assert hasattr(sca._lib, name), name
+
+
+@pytest.mark.parametrize("seg, msg", [
+    (W.Segment(0, 4, 1), "num_frames"),
+    (W.Segment(2, 0, 1), "tokens_per_frame"),
+    (W.Segment(2, 4, -1), "head_len"),
+    (W.Segment(2, 4, 1, (W.Action(3, 1, 1),)), "action 0"),
+    (W.Segment(2, 4, 1, (W.Action(0, 0, 1),)), "action 0"),
+    (W.Segment(2, 4, 1, (W.Action(3, 0, 3),)), "action 0"),
+    (W.Segment(2, 4, 1, tuple(W.Action(1, 0, 1) for _ in range(33))), "num_actions"),
+])
+def test_builder_rejects_bad_layouts(seg, msg):
+    with pytest.raises(sca.ScaError) as e:
+        sca.build_segment_mask_metadata((), (seg,))
+    assert e.value.code == sca.ERR_INVALID_ARG and msg in str(e.value)
+
+
+def test_builder_rejects_empty_current_and_bad_policy():
+    with pytest.raises(sca.ScaError):
+        sca.build_segment_mask_metadata((), ())
+    with pytest.raises(sca.ScaError):
+        sca.build_segment_mask_metadata((), (W.Segment(1, 1, 0),), textq_policy=7)
+
+
+def test_rebuild_replaces_contents():
+    md = sca.build_segment_mask_metadata((), (W.Segment(1, 1, 0),))
+    assert md.counts()["n_queries"] == 1
+    md.build(W.small_session().cached, W.small_session().current)
+    assert md.counts()["n_queries"] == W.small_session().n_query_tokens
