@@ -213,6 +213,24 @@ def run_reference(args, problem):
 # the native arm
 # ---------------------------------------------------------------------------
 
+def reduce_max(x: float, world: int, device: str) -> float:
+    """Max of a per-rank number over all ranks (device times are reported as
+    the slowest rank's)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_step: float, steps: int, max_ms: float) -> float:
+    """Units processed by all ranks divided by the slowest rank's time."""
+    return world * flops_per_step * steps / (max_ms * 1e-3) / 1e12
+
+
 class Session:
     """One replica of the workload on the current device: a cache holding the
     prior segments, the current segment's Q/K/V, outputs and metadata."""
@@ -290,11 +308,7 @@ def run_native(args, problem):
             dist.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, "cuda")
 
     sess = Session(problem, seed=1000 * 2 + rank)
     from segment_causal_masked_b200 import sca
@@ -327,7 +341,7 @@ def run_native(args, problem):
     attn_ms = [a.elapsed_time(b) for a, b in evs]
     attn_avg = max_over_ranks(statistics.mean(attn_ms))
     ms_step = ms_total / args.steps
-    value = world * flops * args.steps / (ms_total * 1e-3) / 1e12
+    value = whole_job_tflops(world, flops, args.steps, ms_total)
 
     # ---- end to end through the API with pinned host buffers
     nq, h = problem.n_query_tokens, problem.heads
@@ -357,7 +371,7 @@ def run_native(args, problem):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = world * flops * args.steps / (e2e_ms * 1e-3) / 1e12
+    e2e_value = whole_job_tflops(world, flops, args.steps, e2e_ms)
     bytes_in = 3 * hq.numel() * hq.element_size()
     bytes_out = ho.numel() * ho.element_size()
 
