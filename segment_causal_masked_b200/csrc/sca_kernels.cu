@@ -148,6 +148,14 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Common case inline; the bounded polling loop only when the phase is not
+// complete yet (keeps the call, and its register spills, off the fast path).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile Ctl* ctl,
+                                         int32_t* status, unsigned long long timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_bounded(bar, parity, ctl, status, timeout_ns);
+}
+
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int32_t c0, int32_t c1, int32_t c2) {
   asm volatile(
@@ -256,6 +264,32 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+  return m;
+}
+
+// Packed fp32 pairs (one instruction for two lanes of work on sm_100).
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void unf2(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -370,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kv = 0; kv < 2; ++kv, ++it) {
           const int s = it % kStages;
           const uint32_t ph = uint32_t(it / kStages) & 1u;
-          if (!wait_bounded(bar(kBarEmpty + s), ph ^ 1u, ctl, p.status, p.timeout_ns)) {
+          if (!wait_bar(bar(kBarEmpty + s), ph ^ 1u, ctl, p.status, p.timeout_ns)) {
             ok = false;
             break;
           }
@@ -418,10 +452,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       auto stage_of = [&](int it) { return sbase + kOffKV + uint32_t(it % kStages) * kTile; };
       auto wait_full = [&](int it) {
-        return wait_bounded(bar(kBarFull + it % kStages), uint32_t(it / kStages) & 1u, ctl,
-                            p.status, p.timeout_ns);
+        return wait_bar(bar(kBarFull + it % kStages), uint32_t(it / kStages) & 1u, ctl, p.status,
+                        p.timeout_ns);
       };
-      bool ok = wait_bounded(bar(kBarQ), 0, ctl, p.status, p.timeout_ns) && wait_full(0);
+      bool ok = wait_bar(bar(kBarQ), 0, ctl, p.status, p.timeout_ns) && wait_full(0);
       if (ok) {
         tc_fence_after();
         issue_qk(tS0, sQ0, stage_of(0));
@@ -434,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int itV = 2 * j + 1, itK = 2 * j + 2;
         const uint32_t ph = uint32_t(j) & 1u;
         const bool more = j + 1 < n_iter;
-        ok = wait_full(itV) && wait_bounded(bar(kBarP + 0), ph, ctl, p.status, p.timeout_ns);
+        ok = wait_full(itV) && wait_bar(bar(kBarP + 0), ph, ctl, p.status, p.timeout_ns);
         if (!ok) break;
         tc_fence_after();
         issue_pv(tO0, tS0, stage_of(itV), j > 0);
@@ -444,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_qk(tS0, sQ0, stage_of(itK));
           mma_commit(bar(kBarS + 0));
         }
-        if (!(ok = wait_bounded(bar(kBarP + 1), ph, ctl, p.status, p.timeout_ns))) break;
+        if (!(ok = wait_bar(bar(kBarP + 1), ph, ctl, p.status, p.timeout_ns))) break;
         tc_fence_after();
         issue_pv(tO1, tS1, stage_of(itV), j > 0);
         mma_commit(bar(kBarEmpty + itV % kStages));
@@ -474,8 +508,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* kds = kdesc_s + t * 128;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
+    const uint64_t scale2 = f2(p.scale_log2, p.scale_log2);
+    uint32_t e_next = n_iter > 0 ? list[0] : 0u;
     for (int j = 0; j < n_iter; ++j) {
-      const uint32_t e = list[j];
+      const uint32_t e = e_next;
+      if (j + 1 < n_iter) e_next = list[j + 1];   // prefetch the next schedule entry
       const int tile = int(e & kPairTileMask);
       const uint32_t cls = (e >> (24 + 2 * t)) & 3u;
       const bool cached = tile < p.n_cache_tiles;
@@ -483,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int key_limit = (cached ? p.n_cache : p.n_q) - key0;  // existing keys in the tile
       uint32_t kd = 0;
       if (cls == SCA_TILE_PARTIAL) kd = cached ? p.kdesc_cache[key0 + r] : p.kdesc_cur[key0 + r];
-      ok = wait_bounded(bar(kBarS + t), uint32_t(j) & 1u, ctl, p.status, p.timeout_ns);
+      ok = wait_bar(bar(kBarS + t), uint32_t(j) & 1u, ctl, p.status, p.timeout_ns);
       if (!__all_sync(0xFFFFFFFFu, ok)) {  // keep the warp's collective TMEM ops uniform
         ok = false;
         break;
@@ -497,21 +534,45 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_st16(tS + uint32_t(c) * 16, z);
       } else {
-        float s[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + uint32_t(c) * 32, s + 32 * c);
-        tmem_wait_ld();
+        // Two passes over the 128 score columns in chunks of 32, the next
+        // chunk's TMEM load in flight while one is processed: registers stay
+        // well under the 168 a thread has at 320 threads per CTA.
+        float ca[32], cb[32];
+        // pass 1: mask (PARTIAL tiles, written back) and row max
         if (cls == SCA_TILE_PARTIAL) {
           kds[r] = kd;
           named_sync(1 + t, 128);
-#pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            if (c >= key_limit || !visible(qd.x, qd.y, kds[c])) s[c] = -INFINITY;
-          }
         }
-        float mx = s[0];
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        auto pass1 = [&](float* x, int c) {
+          if (cls == SCA_TILE_PARTIAL) {
 #pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+            for (int i = 0; i < 32; ++i) {
+              const int col = 32 * c + i;
+              if (col >= key_limit || !visible(qd.x, qd.y, kds[col])) x[i] = -INFINITY;
+            }
+            tmem_st32(tS + uint32_t(c) * 32, x);
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) m4[k] = max3(m4[k], x[i + k], x[i + 4 + k]);
+          }
+        };
+        tmem_ld32(tS, ca);
+        tmem_wait_ld();
+        tmem_ld32(tS + 32, cb);
+        pass1(ca, 0);
+        tmem_wait_ld();
+        tmem_ld32(tS + 64, ca);
+        pass1(cb, 1);
+        tmem_wait_ld();
+        tmem_ld32(tS + 96, cb);
+        pass1(ca, 2);
+        tmem_wait_ld();
+        pass1(cb, 3);
+        if (cls == SCA_TILE_PARTIAL) tmem_wait_st();   // masked scores are back in TMEM
+        const float mx = max3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
         // The running max only moves when it grows by more than the threshold
         // (exact: l and O share the stale max until the final division).
         const float m_cand = mx * p.scale_log2;
@@ -520,42 +581,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float alpha = rescale ? ex2(m_run - m_cand) : 1.f;
         if (grow) m_run = m_cand;
         l_run *= alpha;
-        // tcgen05.ld/st are warp-collective: the whole warp rewrites O if any
-        // row needs it (alpha = 1 for the others). O of earlier tiles was
-        // complete when S of this tile completed (in-order MMA pipeline).
-        if (__any_sync(0xFFFFFFFFu, rescale)) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float o[32];
-            tmem_ld32(tO + uint32_t(c) * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(tO + uint32_t(c) * 32, o);
-          }
-        }
         const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-        float sum = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        const uint64_t negm2 = f2(neg_m, neg_m);
+        uint64_t acc[2] = {0ull, 0ull};  // packed partial sums
+        // pass 2: p = exp2(s * scale_log2 - m), row sum, bf16 P over the first
+        // 64 columns of S (P chunk c lands in S chunk c/2, already consumed)
+        auto pass2 = [&](const float* x, int c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2(fmaf(s[32 * c + 2 * i], p.scale_log2, neg_m));
-            const float p1 = ex2(fmaf(s[32 * c + 2 * i + 1], p.scale_log2, neg_m));
-            sum += p0 + p1;
+            float x0, x1;
+            unf2(fma2(f2(x[2 * i], x[2 * i + 1]), scale2, negm2), x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            acc[i & 1] = add2(acc[i & 1], f2(p0, p1));
             pk[i] = pack_bf16(p0, p1);
           }
           tmem_st16(tS + uint32_t(c) * 16, pk);
+        };
+        tmem_ld32(tS, ca);
+        tmem_wait_ld();
+        tmem_ld32(tS + 32, cb);
+        pass2(ca, 0);
+        tmem_wait_ld();
+        tmem_ld32(tS + 64, ca);
+        pass2(cb, 1);
+        tmem_wait_ld();
+        tmem_ld32(tS + 96, cb);
+        pass2(ca, 2);
+        tmem_wait_ld();
+        pass2(cb, 3);
+        float a0, a1;
+        unf2(add2(acc[0], acc[1]), a0, a1);
+        l_run += a0 + a1;
+        // Rescale O. tcgen05.ld/st are warp-collective: the whole warp
+        // rewrites O if any row needs it (alpha = 1 for the others). O of
+        // earlier tiles was complete when S of this tile completed (in-order
+        // MMA pipeline); P*V of this tile waits for the arrive below.
+        if (__any_sync(0xFFFFFFFFu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            tmem_ld32(tO + uint32_t(c) * 32, ca);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ca[i] *= alpha;
+            tmem_st32(tO + uint32_t(c) * 32, ca);
+          }
         }
-        l_run += sum;
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kBarP + t));
     }
     // ---------------------------------------------------------- epilogue
-    if (ok && n_iter > 0) ok = wait_bounded(bar(kBarO + t), 0, ctl, p.status, p.timeout_ns);
+    if (ok && n_iter > 0) ok = wait_bar(bar(kBarO + t), 0, ctl, p.status, p.timeout_ns);
     if (__all_sync(0xFFFFFFFFu, ok)) {
       tc_fence_after();
       const bool store = q_row < p.n_q;
