@@ -264,6 +264,11 @@ class Session:
         self.lse = torch.empty(h, nq, dtype=torch.float32, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.md = sca.Metadata()
+        self.md.build(problem.cached, problem.current, problem.textq_policy)
+        ws_bytes = sca.attn_workspace_bytes(self.md, h)
+        self.splits = ws_bytes > 0
+        self.plan = sca.attn_plan(self.md, h)
+        self.workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
         self.stream = torch.cuda.current_stream()
         torch.cuda.synchronize()
 
@@ -280,7 +285,7 @@ class Session:
                                    self.k_cur if k_cur is None else k_cur,
                                    self.v_cur if v_cur is None else v_cur,
                                    self.o if o is None else o, self.lse, p.softmax_scale,
-                                   self.status, s)
+                                   self.workspace, None, self.status, s)
         if ev is not None:
             ev[1].record(self.stream)
         self.cache.append(p.current[0], self.k_cur if k_cur is None else k_cur,
@@ -392,7 +397,8 @@ def run_native(args, problem):
                        "step": "metadata build+upload, attention forward, kv_cache_append",
                        "l2": "inputs larger than L2 (cached K/V %.2f GB per tensor)"
                              % (problem.n_cache_tokens * h * 256 / 1e9),
-                       "parallelism": f"replicas x{world}"},
+                       "parallelism": f"replicas x{world}",
+                       "split_plan": sess.plan},
             "pct_of_peak": 100.0 * value / world / peak,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
@@ -400,7 +406,7 @@ def run_native(args, problem):
                          "peak_source": f"{peaks['source']} bf16 dense (burst)"},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": bytes_in,
                     "d2h_bytes_per_step": bytes_out, "ms_per_step": e2e_ms / args.steps},
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": (2 + (1 if sess.splits else 0)) * args.steps,
             "clocks": clock_info,
         }
         if not args.no_cpu_baseline:

@@ -206,15 +206,37 @@ SCA_API void sca_kv_cache_destroy(sca_kv_cache* cache);
  *   md     : built and uploaded (sca_metadata_upload) before this call;
  *   q, k_cur, v_cur, o : bf16 token-major [n_queries][heads][128];
  *   lse    : fp32 [heads][n_queries] natural-log sum-exp, or NULL;
+ *   workspace, workspace_bytes : optional device scratch (256-byte aligned).
+ *            With enough of it (sca_attn_workspace_bytes) the work items
+ *            left after the last full wave of SMs are split along the keys
+ *            and merged by a second kernel, which removes the partial last
+ *            wave; with NULL or too little, nothing is split. The result is
+ *            the same up to fp32 summation order;
  *   dev_status : device int32 (or NULL); left unchanged on success, set to
  *            SCA_ERR_DEVICE_TIMEOUT if a bounded wait in the kernel ran out;
  *   stream : the caller's stream.
  * The call allocates nothing. A query that sees no key gets o = 0 and
- * lse = -inf. */
+ * lse = -inf. Calls sharing a workspace must be ordered (same stream). */
 SCA_API int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md,
                                int32_t heads, const void* q, const void* k_cur,
                                const void* v_cur, void* o, float* lse,
-                               float softmax_scale, int32_t* dev_status, void* stream);
+                               float softmax_scale, void* workspace, uint64_t workspace_bytes,
+                               int32_t* dev_status, void* stream);
+
+/* Workspace the attention would use on the current device for `heads` heads
+ * (0 when the plan splits nothing). */
+SCA_API int sca_attn_workspace_bytes(const sca_metadata* md, int32_t heads, uint64_t* bytes);
+
+/* The plan the next attention call with enough workspace would run: the
+ * first n_full work items (query-tile pair x head) whole, the remaining
+ * n_split items cut into `chunks` key ranges each. Any output may be NULL. */
+SCA_API int sca_attn_plan(const sca_metadata* md, int32_t heads, int32_t* n_full,
+                          int32_t* n_split, int32_t* chunks);
+
+/* Process-wide override of the key-split factor used by later attention calls:
+ * 0 = automatic (default), 1 = never split, k >= 2 = split every work item
+ * after the full waves into k chunks (a test and tuning knob). */
+SCA_API int sca_set_split_override(int32_t chunks);
 
 /* Message of the calling thread's last failure ("" if none). */
 SCA_API const char* sca_last_error(void);
@@ -226,6 +248,12 @@ SCA_API const char* sca_last_error(void);
  * path can be exercised without any real hang.
  * ------------------------------------------------------------------------- */
 SCA_API int sca_debug_bounded_wait(int32_t* dev_status, int64_t timeout_ns, void* stream);
+
+/* Evaluate, for n floats x (device, x <= 8), the two exponentials the
+ * attention kernel uses: y_poly = 2^x by range reduction and a fitted cubic
+ * on the FMA pipe, y_mufu = 2^x by the ex2.approx instruction. For testing
+ * the first against the second and against float64. */
+SCA_API int sca_debug_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n, void* stream);
 
 #ifdef __cplusplus
 }

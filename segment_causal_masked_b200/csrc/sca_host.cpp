@@ -9,12 +9,15 @@
 // words, the same predicate the attention kernel applies on PARTIAL tiles.
 
 #include <math.h>
+
+#include <cmath>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
 
 #include <algorithm>
 #include <numeric>
+#include <queue>
 
 #include "sca_internal.h"
 
@@ -277,6 +280,27 @@ int sca_build_segment_mask_metadata(sca_metadata* md, const sca_segment* cached,
       return fail(SCA_ERR_UNSUPPORTED, "schedule larger than 2^31 entries");
   }
 
+  // --- runs of equal descriptors inside each key tile (for the kernel's
+  // per-row visibility masks on PARTIAL tiles) ---------------------------
+  std::vector<int32_t> run_ptr(size_t(n_ct + n_ut) + 1, 0);
+  std::vector<uint32_t> runs;
+  auto add_runs = [&](const std::vector<uint32_t>& d, int64_t n, int64_t tile0) {
+    for (int64_t t = 0; t * SCA_TILE < n; ++t) {
+      const int64_t k0 = t * SCA_TILE, k1 = std::min<int64_t>(n, k0 + SCA_TILE);
+      int64_t a = k0;
+      while (a < k1) {
+        int64_t b = a + 1;
+        while (b < k1 && d[size_t(b)] == d[size_t(a)]) ++b;
+        runs.push_back(uint32_t(a - k0) | (uint32_t(b - a) << 8));
+        runs.push_back(d[size_t(a)]);
+        a = b;
+      }
+      run_ptr[size_t(tile0 + t) + 1] = int32_t(runs.size() / 2);
+    }
+  };
+  add_runs(kdesc_cache, n_cache, 0);
+  add_runs(kdesc_cur, n_q, n_ct);
+
   // --- kernel work list: query-tile pairs, union of their key tiles --------
   const int n_pairs = (n_qt + 1) / 2;
   std::vector<int32_t> pair_ptr(size_t(n_pairs) + 1, 0);
@@ -297,14 +321,26 @@ int sca_build_segment_mask_metadata(sca_metadata* md, const sca_segment* cached,
     }
     pair_ptr[size_t(p) + 1] = int32_t(pair_list.size());
   }
+  // Estimated cost of a pair, in (query tile x key tile) units: a FULL tile
+  // is one unit, a PARTIAL one a little more (its mask), an EMPTY one only
+  // the shared loads and handshakes (the kernel skips its MMAs and softmax).
+  std::vector<float> pair_cost((size_t)n_pairs, 0.f);
+  const float w_cls[4] = {0.1f, 1.25f, 1.f, 0.f};
+  for (int p = 0; p < n_pairs; ++p) {
+    float c = 0.f;
+    for (int32_t i = pair_ptr[size_t(p)]; i < pair_ptr[size_t(p) + 1]; ++i)
+      c += w_cls[(pair_list[size_t(i)] >> 24) & 3u] + w_cls[(pair_list[size_t(i)] >> 26) & 3u];
+    pair_cost[size_t(p)] = c;
+  }
   std::vector<int32_t> order((size_t)n_pairs);
   std::iota(order.begin(), order.end(), 0);
   std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
-    return pair_ptr[size_t(x) + 1] - pair_ptr[size_t(x)] > pair_ptr[size_t(y) + 1] - pair_ptr[size_t(y)];
+    return pair_cost[size_t(x)] > pair_cost[size_t(y)];
   });
 
   md->built = true;
   md->uploaded = false;
+  md->plan_key[0] = -1;
   md->n_cached = n_cached;
   md->n_current = n_current;
   md->policy = policy;
@@ -326,6 +362,9 @@ int sca_build_segment_mask_metadata(sca_metadata* md, const sca_segment* cached,
   md->pair_ptr.swap(pair_ptr);
   md->pair_list.swap(pair_list);
   md->item_order.swap(order);
+  md->pair_cost.swap(pair_cost);
+  md->run_ptr.swap(run_ptr);
+  md->runs.swap(runs);
   return SCA_OK;
 }
 
@@ -370,13 +409,13 @@ int sca_metadata_upload(sca_metadata* md, void* stream) {
   if (int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
   // layout of the device block
   const size_t nq_pad = size_t(md->n_pairs) * 2 * SCA_TILE;
-  const size_t nk_pad = align_up(size_t(md->n_q), SCA_TILE);
   size_t off = 0;
   const size_t off_q = off;     off = align_up(off + nq_pad * 8, 256);
-  const size_t off_k = off;     off = align_up(off + nk_pad * 4, 256);
   const size_t off_o = off;     off = align_up(off + size_t(md->n_pairs) * 4, 256);
   const size_t off_p = off;     off = align_up(off + (size_t(md->n_pairs) + 1) * 4, 256);
   const size_t off_l = off;     off = align_up(off + std::max<size_t>(md->pair_list.size(), 1) * 4, 256);
+  const size_t off_rp = off;    off = align_up(off + md->run_ptr.size() * 4, 256);
+  const size_t off_r = off;     off = align_up(off + std::max<size_t>(md->runs.size(), 2) * 4, 256);
   const size_t bytes = off;
 
   if (md->upload_done) {  // the staging buffer may still feed the previous copy
@@ -405,21 +444,21 @@ int sca_metadata_upload(sca_metadata* md, void* stream) {
   uint8_t* h = static_cast<uint8_t*>(md->pinned);
   memset(h, 0, bytes);
   memcpy(h + off_q, md->query_desc.data(), md->query_desc.size() * 4);  // padding: invalid queries
-  uint32_t* kd = reinterpret_cast<uint32_t*>(h + off_k);
-  memcpy(kd, md->key_desc_cur.data(), md->key_desc_cur.size() * 4);
-  for (size_t i = md->key_desc_cur.size(); i < nk_pad; ++i) kd[i] = SCA_DESC_SEG_MASK;  // never visible
   memcpy(h + off_o, md->item_order.data(), md->item_order.size() * 4);
   memcpy(h + off_p, md->pair_ptr.data(), md->pair_ptr.size() * 4);
   memcpy(h + off_l, md->pair_list.data(), md->pair_list.size() * 4);
+  memcpy(h + off_rp, md->run_ptr.data(), md->run_ptr.size() * 4);
+  memcpy(h + off_r, md->runs.data(), md->runs.size() * 4);
   if (int rc = check_cuda(cudaMemcpyAsync(md->dev, h, bytes, cudaMemcpyHostToDevice, st),
                           "cudaMemcpyAsync(metadata)"))
     return rc;
   if (int rc = check_cuda(cudaEventRecord(md->upload_done, st), "cudaEventRecord")) return rc;
   md->off_qdesc = off_q;
-  md->off_kdesc = off_k;
   md->off_order = off_o;
   md->off_ptr = off_p;
   md->off_list = off_l;
+  md->off_run_ptr = off_rp;
+  md->off_runs = off_r;
   md->uploaded = true;
   return SCA_OK;
 }
@@ -549,10 +588,133 @@ static int make_map(CUtensorMap* m, const void* base, uint64_t dim1, uint64_t di
   return SCA_OK;
 }
 
+// ---------------------------------------------------------------------------
+// work split across the SMs
+// ---------------------------------------------------------------------------
+
+static int g_split_override = 0;
+
+static int device_sms(int dev) {
+  static int cached[64] = {0};
+  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  int sms = 148;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;
+  if (dev >= 0 && dev < 64) cached[dev] = sms;
+  return sms;
+}
+
+// Work items are (query-tile pair, head), most expensive pair first, heads
+// inner; one CTA runs one item (or one chunk of one). The plan keeps the
+// first `n_full` items whole and cuts each of the remaining `n_split` items
+// into `chunks` key ranges, so the last wave of SMs is not left half empty. It
+// is chosen by simulating greedy dispatch of the CTAs in launch order onto the
+// SMs (one CTA per SM), with the pairs' estimated costs plus fixed per-CTA
+// and per-split overheads, over a few candidate plans.
+static void choose_plan(const sca_metadata* md, int heads, int sms, int forced,
+                        int32_t* n_full, int32_t* n_split, int32_t* chunks) {
+  const int64_t N = int64_t(md->n_pairs) * heads;
+  auto len = [&](int64_t item) {
+    return double(md->pair_cost[size_t(md->item_order[size_t(item / heads)])]);
+  };
+  const double c_cta = 4.0, c_split = 4.0;  // per-CTA start-up; partial store + merge
+  auto makespan = [&](int64_t nf, int k) {
+    std::priority_queue<double, std::vector<double>, std::greater<double>> q;
+    for (int i = 0; i < sms; ++i) q.push(0.0);
+    auto run = [&](double cost) {
+      const double t = q.top();
+      q.pop();
+      q.push(t + cost);
+    };
+    for (int64_t i = 0; i < nf; ++i) run(len(i) + c_cta);
+    for (int c = 0; c < k; ++c)
+      for (int64_t i = nf; i < N; ++i) run(std::ceil(len(i) / k) + c_cta + c_split);
+    double m = 0;
+    while (!q.empty()) {
+      m = std::max(m, q.top());
+      q.pop();
+    }
+    return m;
+  };
+  *n_full = int32_t(N);
+  *n_split = 0;
+  *chunks = 1;
+  if (forced == 1 || N == 0) return;
+  const int64_t waves = N / sms;
+  if (forced >= 2) {
+    const int64_t nf = waves >= 1 ? (waves - 1) * sms : 0;
+    *n_full = int32_t(nf);
+    *n_split = int32_t(N - nf);
+    *chunks = forced;
+    return;
+  }
+  double best = makespan(N, 1);
+  const int64_t cands[3] = {waves >= 2 ? (waves - 2) * sms : 0, waves >= 1 ? (waves - 1) * sms : 0,
+                            waves * sms};
+  const int ks[6] = {2, 3, 4, 5, 6, 8};
+  for (int64_t nf : cands) {
+    if (nf >= N) continue;
+    for (int k : ks) {
+      const double m = makespan(nf, k);
+      if (m < best * 0.995) {  // splitting has to pay for itself
+        best = m;
+        *n_full = int32_t(nf);
+        *n_split = int32_t(N - nf);
+        *chunks = k;
+      }
+    }
+  }
+}
+
+static void plan_for(const sca_metadata* md, int heads, int dev) {
+  const int sms = device_sms(dev);
+  if (md->plan_key[0] == heads && md->plan_key[1] == sms && md->plan_key[2] == g_split_override &&
+      md->plan_key[3] == dev)
+    return;
+  int32_t nf, ns, k;
+  choose_plan(md, heads, sms, g_split_override, &nf, &ns, &k);
+  md->plan_full = nf;
+  md->plan_split = ns;
+  md->plan_chunks = k;
+  md->plan_ws = k > 1 ? uint64_t(ns) * uint64_t(k) * kPartialSlotBytes : 0;
+  md->plan_key[0] = heads;
+  md->plan_key[1] = sms;
+  md->plan_key[2] = g_split_override;
+  md->plan_key[3] = dev;
+}
+
+int sca_set_split_override(int32_t chunks) {
+  if (chunks < 0 || chunks > 64) return fail(SCA_ERR_INVALID_ARG, "split override must be in [0, 64]");
+  g_split_override = chunks;
+  return SCA_OK;
+}
+
+int sca_attn_workspace_bytes(const sca_metadata* md, int32_t heads, uint64_t* bytes) {
+  if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
+  if (heads < 1 || !bytes) return fail(SCA_ERR_INVALID_ARG, "need heads >= 1 and an output pointer");
+  int dev = 0;
+  if (int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
+  plan_for(md, heads, dev);
+  *bytes = md->plan_ws;
+  return SCA_OK;
+}
+
+int sca_attn_plan(const sca_metadata* md, int32_t heads, int32_t* n_full, int32_t* n_split,
+                  int32_t* chunks) {
+  if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
+  if (heads < 1) return fail(SCA_ERR_INVALID_ARG, "need heads >= 1");
+  int dev = 0;
+  if (int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
+  plan_for(md, heads, dev);
+  if (n_full) *n_full = md->plan_full;
+  if (n_split) *n_split = md->plan_split;
+  if (chunks) *chunks = md->plan_chunks;
+  return SCA_OK;
+}
+
 int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md, int32_t heads,
                                const void* q, const void* k_cur, const void* v_cur, void* o,
-                               float* lse, float softmax_scale, int32_t* dev_status,
-                               void* stream) {
+                               float* lse, float softmax_scale, void* workspace,
+                               uint64_t workspace_bytes, int32_t* dev_status, void* stream) {
   if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
   if (!md->uploaded) return fail(SCA_ERR_INVALID_ARG, "metadata not uploaded");
   if (heads < 1) return fail(SCA_ERR_INVALID_ARG, "heads must be >= 1");
@@ -560,6 +722,8 @@ int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md
   if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(o) ||
       (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
     return fail(SCA_ERR_MISALIGNED, "q, k_cur, v_cur, o must be 16-byte aligned (lse 4-byte)");
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(SCA_ERR_MISALIGNED, "workspace must be 256-byte aligned");
   if (!(softmax_scale > 0.f) || !isfinite(softmax_scale))
     return fail(SCA_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
   if (md->n_cached > 0) {
@@ -575,7 +739,7 @@ int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md
   int dev = 0;
   if (int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
   if (dev != md->device) return fail(SCA_ERR_MISMATCH, "metadata was uploaded to another device");
-  if (int64_t(md->n_pairs) * heads > INT32_MAX) return fail(SCA_ERR_UNSUPPORTED, "grid too large");
+  if (int64_t(md->n_pairs) * heads * 64 > INT32_MAX) return fail(SCA_ERR_UNSUPPORTED, "grid too large");
 
   const uint64_t row = uint64_t(heads) * SCA_HEAD_DIM * 2;  // bytes per token, token-major
   AttnMaps maps;
@@ -592,14 +756,15 @@ int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md
   }
   if (rc) return rc;
 
+  plan_for(md, heads, dev);
   const uint8_t* d = static_cast<const uint8_t*>(md->dev);
   AttnArgs a{};
   a.qdesc = reinterpret_cast<const uint2*>(d + md->off_qdesc);
-  a.kdesc_cur = reinterpret_cast<const uint32_t*>(d + md->off_kdesc);
-  a.kdesc_cache = md->n_cache > 0 ? cache->desc : nullptr;
   a.item_order = reinterpret_cast<const int32_t*>(d + md->off_order);
   a.pair_ptr = reinterpret_cast<const int32_t*>(d + md->off_ptr);
   a.pair_list = reinterpret_cast<const uint32_t*>(d + md->off_list);
+  a.run_ptr = reinterpret_cast<const int32_t*>(d + md->off_run_ptr);
+  a.runs = reinterpret_cast<const uint2*>(d + md->off_runs);
   a.o = o;
   a.lse = lse;
   a.status = dev_status;
@@ -610,8 +775,27 @@ int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md
   a.n_pairs = md->n_pairs;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.timeout_ns = 2000000000ull;
-  return check_cuda(launch_attention(maps, a, static_cast<cudaStream_t>(stream)),
-                    "attention launch");
+  const bool split = md->plan_chunks > 1 && workspace && workspace_bytes >= md->plan_ws;
+  a.n_full = split ? md->plan_full : md->n_pairs * heads;
+  a.n_split = split ? md->plan_split : 0;
+  a.chunks = split ? md->plan_chunks : 1;
+  if (split) {
+    const uint64_t slots = uint64_t(a.n_split) * uint64_t(a.chunks);
+    a.part_o = static_cast<float*>(workspace);
+    a.part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + slots * 256 * 128 * 4);
+  }
+  if (int rc2 = check_cuda(launch_attention(maps, a, static_cast<cudaStream_t>(stream)),
+                           "attention launch"))
+    return rc2;
+  if (split)
+    return check_cuda(launch_merge(a, static_cast<cudaStream_t>(stream)), "merge launch");
+  return SCA_OK;
+}
+
+int sca_debug_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n, void* stream) {
+  if (!x || !y_poly || !y_mufu || n < 0) return fail(SCA_ERR_INVALID_ARG, "bad exp2 arguments");
+  return check_cuda(launch_exp2_eval(x, y_poly, y_mufu, n, static_cast<cudaStream_t>(stream)),
+                    "exp2 launch");
 }
 
 int sca_debug_bounded_wait(int32_t* dev_status, int64_t timeout_ns, void* stream) {

@@ -57,15 +57,24 @@ constexpr uint32_t kPairTileMask = 0xFFFFFFu;
 struct AttnArgs {
   // metadata (device)
   const uint2* qdesc;          // [n_pairs * 256]
-  const uint32_t* kdesc_cur;   // [round_up(n_q, 128)]
-  const uint32_t* kdesc_cache; // [round_up(capacity, 128)] or null
   const int32_t* item_order;   // [n_pairs] longest list first
   const int32_t* pair_ptr;     // [n_pairs + 1]
   const uint32_t* pair_list;   // [pair_ptr[n_pairs]]
+  const int32_t* run_ptr;      // [n_kv_tiles + 1] runs of each key tile
+  const uint2* runs;           // {first column | count << 8, key descriptor}
   // outputs
   void* o;                     // bf16 [n_q][heads][128]
   float* lse;                  // [heads][n_q] or null
   int32_t* status;             // device status word or null
+  // split-KV tail: CTAs [0, n_full) run whole items; the next
+  // n_split * chunks CTAs run chunk k of item n_full + si (chunk-major) and
+  // write fp32 partials (unnormalised O, running max and sum, log2 domain)
+  // to slot si * chunks + k
+  float* part_o;               // [slots][256][128]
+  float2* part_ml;             // [slots][256]
+  int32_t n_full;
+  int32_t n_split;
+  int32_t chunks;
   // sizes
   int32_t n_q;
   int32_t n_cache;             // cache keys
@@ -81,6 +90,10 @@ struct AttnMaps {
 };
 
 cudaError_t launch_attention(const AttnMaps& maps, const AttnArgs& args, cudaStream_t stream);
+cudaError_t launch_merge(const AttnArgs& args, cudaStream_t stream);
+
+// bytes of one partial slot: O [256][128] fp32 + (m, l) [256]
+constexpr uint64_t kPartialSlotBytes = 256ull * 128 * 4 + 256ull * 8;
 
 struct AppendArgs {
   const void* k;
@@ -102,6 +115,8 @@ struct AppendArgs {
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
 cudaError_t launch_bounded_wait(int32_t* status, unsigned long long timeout_ns,
                                 cudaStream_t stream);
+cudaError_t launch_exp2_eval(const float* x, float* y_poly, float* y_mufu, int64_t n,
+                             cudaStream_t stream);
 
 size_t attention_smem_bytes();
 
@@ -128,7 +143,10 @@ struct sca_metadata {
   std::vector<uint8_t> flag;           // [nnz]
   std::vector<int32_t> pair_ptr;       // [n_pairs + 1]
   std::vector<uint32_t> pair_list;
-  std::vector<int32_t> item_order;     // [n_pairs]
+  std::vector<int32_t> item_order;     // [n_pairs], most expensive first
+  std::vector<float> pair_cost;        // [n_pairs] estimated cost (query-tile x key-tile units)
+  std::vector<int32_t> run_ptr;        // [n_kv_tiles + 1]
+  std::vector<uint32_t> runs;          // pairs of words: first | count << 8, descriptor
   // device copy
   bool uploaded = false;
   int device = -1;
@@ -137,7 +155,12 @@ struct sca_metadata {
   void* pinned = nullptr;
   size_t pinned_bytes = 0;
   cudaEvent_t upload_done = nullptr;
-  size_t off_qdesc = 0, off_kdesc = 0, off_order = 0, off_ptr = 0, off_list = 0;
+  size_t off_qdesc = 0, off_order = 0, off_ptr = 0, off_list = 0;
+  size_t off_run_ptr = 0, off_runs = 0;
+  // last split plan (heads, SMs, workspace, override) -> plan
+  mutable int32_t plan_key[4] = {-1, -1, -1, -1};
+  mutable uint64_t plan_ws = 0;
+  mutable int32_t plan_full = 0, plan_split = 0, plan_chunks = 1;
 };
 
 struct sca_kv_cache {

@@ -292,6 +292,34 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   return r;
 }
 
+// 2^x on the FMA pipe, for finite x <= 8 (Cody-Waite range reduction):
+// x = j + f with j = rint(x) and f in [-1/2, 1/2]; 2^f from a cubic fitted
+// for minimax relative error on [-1/2, 1/2] by csrc/fit_exp2.py (Remez
+// exchange, 7.5e-5 after rounding the coefficients to float32); 2^j is added
+// to the exponent field. x is clamped at -126 so the exponent stays in range;
+// below that the result is a negligible value near 2^-126 (not 0), so this is
+// only used where no score is -inf (FULL tiles).
+constexpr float kExp2C0 = 0x1.fff692p-1f;
+constexpr float kExp2C1 = 0x1.62f31ap-1f;
+constexpr float kExp2C2 = 0x1.f0de1ap-3f;
+constexpr float kExp2C3 = 0x1.c3f76p-5f;
+constexpr float kRoundMagic = 12582912.f;  // 1.5 * 2^23: adding it leaves rint(x) in the low bits
+
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  const uint64_t x = f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = add2(x, f2(kRoundMagic, kRoundMagic));
+  const uint64_t j = add2(t, f2(-kRoundMagic, -kRoundMagic));
+  const uint64_t f = fma2(j, f2(-1.f, -1.f), x);
+  uint64_t p = fma2(f2(kExp2C3, kExp2C3), f, f2(kExp2C2, kExp2C2));
+  p = fma2(p, f, f2(kExp2C1, kExp2C1));
+  p = fma2(p, f, f2(kExp2C0, kExp2C0));
+  float p0, p1, t0, t1;
+  unf2(p, p0, p1);
+  unf2(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -321,12 +349,12 @@ constexpr int kMmaWarp = 9;
 constexpr uint32_t kHalf = 128 * 64 * 2;  // one 128-row x 64-column bf16 box: 16 KB
 constexpr uint32_t kTile = 2 * kHalf;     // 128 x 128 bf16: 32 KB
 constexpr float kRescaleThreshold = 8.0f; // log2 units: p stays <= 2^8 between rescales
+constexpr int kPolyEvery = 4;             // 1 in 4 exponential pairs on the FMA pipe (FULL tiles)
 
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr uint32_t kOffQ = 0;                            // Q0, Q1
 constexpr uint32_t kOffKV = 2 * kTile;                   // ring of K/V tiles
-constexpr uint32_t kOffDesc = kOffKV + kStages * kTile;  // 2 x 128 key descriptors
-constexpr uint32_t kOffBar = kOffDesc + 2 * 128 * 4;
+constexpr uint32_t kOffBar = kOffKV + kStages * kTile;
 constexpr uint32_t kBarQ = 0, kBarFull = 1, kBarEmpty = kBarFull + kStages,
                    kBarS = kBarEmpty + kStages, kBarP = kBarS + 2, kBarO = kBarP + 2,
                    kBarDrain = kBarO + 2, kNumBars = kBarDrain + 1;
@@ -350,15 +378,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](uint32_t i) { return bar0 + 8 * i; };
   volatile Ctl* ctl = reinterpret_cast<volatile Ctl*>(smem + kOffCtl);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffTmemSlot);
-  uint32_t* kdesc_s = reinterpret_cast<uint32_t*>(smem + kOffDesc);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rank = blockIdx.x / p.heads;
-  const int head = blockIdx.x - rank * p.heads;
+  // which work item (query-tile pair x head), and which of its key tiles
+  int item = int(blockIdx.x), chunk = 0, slot = -1;
+  if (item >= p.n_full) {  // a key chunk of a split item (chunk-major order)
+    const int u = item - p.n_full;
+    chunk = u / p.n_split;
+    const int si = u - chunk * p.n_split;
+    item = p.n_full + si;
+    slot = si * p.chunks + chunk;
+  }
+  const int rank = item / p.heads;
+  const int head = item - rank * p.heads;
   const int pair = p.item_order[rank];
-  const int list_begin = p.pair_ptr[pair];
-  const int n_iter = p.pair_ptr[pair + 1] - list_begin;
-  const uint32_t* list = p.pair_list + list_begin;
+  const int pair_len = p.pair_ptr[pair + 1] - p.pair_ptr[pair];
+  const int j_begin = int((int64_t(pair_len) * chunk) / p.chunks);
+  const int j_end = slot < 0 ? pair_len : int((int64_t(pair_len) * (chunk + 1)) / p.chunks);
+  const int n_iter = j_end - j_begin;
+  const uint32_t* list = p.pair_list + p.pair_ptr[pair] + j_begin;
   const int q_row0 = pair * 256;
 
   if (threadIdx.x == 0) {
@@ -455,12 +493,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         return wait_bar(bar(kBarFull + it % kStages), uint32_t(it / kStages) & 1u, ctl, p.status,
                         p.timeout_ns);
       };
+      // a tile of the pair that sees nothing of key tile j gets neither its
+      // S nor its P V; its barriers still complete (a commit with nothing
+      // new arrives once the earlier MMAs are done)
+      auto live = [&](int j, int t) { return ((list[j] >> (24 + 2 * t)) & 3u) != SCA_TILE_EMPTY; };
+      bool acc0 = false, acc1 = false;  // has O_t received a P V yet
       bool ok = wait_bar(bar(kBarQ), 0, ctl, p.status, p.timeout_ns) && wait_full(0);
       if (ok) {
         tc_fence_after();
-        issue_qk(tS0, sQ0, stage_of(0));
+        if (live(0, 0)) issue_qk(tS0, sQ0, stage_of(0));
         mma_commit(bar(kBarS + 0));
-        issue_qk(tS1, sQ1, stage_of(0));
+        if (live(0, 1)) issue_qk(tS1, sQ1, stage_of(0));
         mma_commit(bar(kBarS + 1));
         mma_commit(bar(kBarEmpty + 0));
       }
@@ -471,19 +514,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_full(itV) && wait_bar(bar(kBarP + 0), ph, ctl, p.status, p.timeout_ns);
         if (!ok) break;
         tc_fence_after();
-        issue_pv(tO0, tS0, stage_of(itV), j > 0);
+        if (live(j, 0)) {
+          issue_pv(tO0, tS0, stage_of(itV), acc0);
+          acc0 = true;
+        }
         if (more) {
           if (!(ok = wait_full(itK))) break;
           tc_fence_after();
-          issue_qk(tS0, sQ0, stage_of(itK));
+          if (live(j + 1, 0)) issue_qk(tS0, sQ0, stage_of(itK));
           mma_commit(bar(kBarS + 0));
         }
         if (!(ok = wait_bar(bar(kBarP + 1), ph, ctl, p.status, p.timeout_ns))) break;
         tc_fence_after();
-        issue_pv(tO1, tS1, stage_of(itV), j > 0);
+        if (live(j, 1)) {
+          issue_pv(tO1, tS1, stage_of(itV), acc1);
+          acc1 = true;
+        }
         mma_commit(bar(kBarEmpty + itV % kStages));
         if (more) {
-          issue_qk(tS1, sQ1, stage_of(itK));
+          if (live(j + 1, 1)) issue_qk(tS1, sQ1, stage_of(itK));
           mma_commit(bar(kBarS + 1));
           mma_commit(bar(kBarEmpty + itK % kStages));
         }
@@ -505,8 +554,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
     const uint32_t tS = lane_base + uint32_t(t) * 128;
     const uint32_t tO = lane_base + 256 + uint32_t(t) * 128;
-    uint32_t* kds = kdesc_s + t * 128;
     float m_run = -INFINITY, l_run = 0.f;
+    bool o_init = false;  // O_t holds a P V result (else its TMEM is undefined)
     bool ok = true;
     const uint64_t scale2 = f2(p.scale_log2, p.scale_log2);
     uint32_t e_next = n_iter > 0 ? list[0] : 0u;
@@ -515,11 +564,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (j + 1 < n_iter) e_next = list[j + 1];   // prefetch the next schedule entry
       const int tile = int(e & kPairTileMask);
       const uint32_t cls = (e >> (24 + 2 * t)) & 3u;
-      const bool cached = tile < p.n_cache_tiles;
-      const int key0 = (cached ? tile : tile - p.n_cache_tiles) * 128;
-      const int key_limit = (cached ? p.n_cache : p.n_q) - key0;  // existing keys in the tile
-      uint32_t kd = 0;
-      if (cls == SCA_TILE_PARTIAL) kd = cached ? p.kdesc_cache[key0 + r] : p.kdesc_cur[key0 + r];
+      // PARTIAL: this row's visibility of the tile's 128 columns, one
+      // predicate per run of equal key descriptors (computed before waiting
+      // for S so it overlaps the MMA); columns past the source are in no run.
+      uint32_t vis[4] = {0u, 0u, 0u, 0u};
+      if (cls == SCA_TILE_PARTIAL) {
+        const int r0 = p.run_ptr[tile], r1 = p.run_ptr[tile + 1];
+        for (int i = r0; i < r1; ++i) {
+          const uint2 run = p.runs[i];
+          if (!visible(qd.x, qd.y, run.y)) continue;
+          const int a = int(run.x & 255u), b = a + int((run.x >> 8) & 255u);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int lo = max(a, 32 * w) - 32 * w, hi = min(b, 32 * w + 32) - 32 * w;
+            if (lo < hi) vis[w] |= uint32_t(((1ull << (hi - lo)) - 1ull) << lo);
+          }
+        }
+      }
       ok = wait_bar(bar(kBarS + t), uint32_t(j) & 1u, ctl, p.status, p.timeout_ns);
       if (!__all_sync(0xFFFFFFFFu, ok)) {  // keep the warp's collective TMEM ops uniform
         ok = false;
@@ -527,89 +588,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       if (cls == SCA_TILE_EMPTY) {
-        // nothing visible for this tile: P = 0
-        uint32_t z[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) z[i] = 0u;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_st16(tS + uint32_t(c) * 16, z);
+        // this tile sees nothing of key tile j: the MMA warp issued neither
+        // its S nor its P V, nothing to do but keep the handshake
       } else {
-        // Two passes over the 128 score columns in chunks of 32, the next
-        // chunk's TMEM load in flight while one is processed: registers stay
-        // well under the 168 a thread has at 320 threads per CTA.
-        float ca[32], cb[32];
-        // pass 1: mask (PARTIAL tiles, written back) and row max
+        // One pass: all 128 scores of the row come out of TMEM with four
+        // loads in flight and a single wait.
+        float x[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + uint32_t(c) * 32, x + 32 * c);
+        tmem_wait_ld();
         if (cls == SCA_TILE_PARTIAL) {
-          kds[r] = kd;
-          named_sync(1 + t, 128);
+#pragma unroll
+          for (int i = 0; i < 128; ++i) x[i] = ((vis[i >> 5] >> (i & 31)) & 1u) ? x[i] : -INFINITY;
         }
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        auto pass1 = [&](float* x, int c) {
-          if (cls == SCA_TILE_PARTIAL) {
+        float m4[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int col = 32 * c + i;
-              if (col >= key_limit || !visible(qd.x, qd.y, kds[col])) x[i] = -INFINITY;
-            }
-            tmem_st32(tS + uint32_t(c) * 32, x);
-          }
+        for (int i = 4; i < 128; i += 8) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) m4[k] = max3(m4[k], x[i + k], x[i + 4 + k]);
-          }
-        };
-        tmem_ld32(tS, ca);
-        tmem_wait_ld();
-        tmem_ld32(tS + 32, cb);
-        pass1(ca, 0);
-        tmem_wait_ld();
-        tmem_ld32(tS + 64, ca);
-        pass1(cb, 1);
-        tmem_wait_ld();
-        tmem_ld32(tS + 96, cb);
-        pass1(ca, 2);
-        tmem_wait_ld();
-        pass1(cb, 3);
-        if (cls == SCA_TILE_PARTIAL) tmem_wait_st();   // masked scores are back in TMEM
+          for (int k = 0; k < 4; ++k) m4[k] = max3(m4[k], x[i + k], x[i + 4 + k]);
+        }
         const float mx = max3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
         // The running max only moves when it grows by more than the threshold
         // (exact: l and O share the stale max until the final division).
         const float m_cand = mx * p.scale_log2;
         const bool grow = m_cand > m_run + kRescaleThreshold;
-        const bool rescale = grow && m_run != -INFINITY && j > 0;
+        const bool rescale = grow && m_run != -INFINITY && o_init;
         const float alpha = rescale ? ex2(m_run - m_cand) : 1.f;
         if (grow) m_run = m_cand;
         l_run *= alpha;
         const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
         const uint64_t negm2 = f2(neg_m, neg_m);
         uint64_t acc[2] = {0ull, 0ull};  // packed partial sums
-        // pass 2: p = exp2(s * scale_log2 - m), row sum, bf16 P over the first
-        // 64 columns of S (P chunk c lands in S chunk c/2, already consumed)
-        auto pass2 = [&](const float* x, int c) {
+        // p = exp2(s * scale_log2 - m), row sum, bf16 P over the first 64
+        // columns of S (all of S is in registers already). On FULL tiles (no
+        // -inf) every kPolyEvery-th pair goes to the FMA pipe instead of the
+        // MUFU, which at d = 128 is otherwise as busy as the tensor cores.
+        const bool full_tile = cls == SCA_TILE_FULL;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            float x0, x1;
-            unf2(fma2(f2(x[2 * i], x[2 * i + 1]), scale2, negm2), x0, x1);
-            const float p0 = ex2(x0), p1 = ex2(x1);
+            float x0, x1, p0, p1;
+            unf2(fma2(f2(x[32 * c + 2 * i], x[32 * c + 2 * i + 1]), scale2, negm2), x0, x1);
+            if (kPolyEvery > 0 && (i % kPolyEvery) == kPolyEvery - 1 && full_tile) {
+              exp2_poly2(x0, x1, p0, p1);
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
             acc[i & 1] = add2(acc[i & 1], f2(p0, p1));
             pk[i] = pack_bf16(p0, p1);
           }
           tmem_st16(tS + uint32_t(c) * 16, pk);
-        };
-        tmem_ld32(tS, ca);
-        tmem_wait_ld();
-        tmem_ld32(tS + 32, cb);
-        pass2(ca, 0);
-        tmem_wait_ld();
-        tmem_ld32(tS + 64, ca);
-        pass2(cb, 1);
-        tmem_wait_ld();
-        tmem_ld32(tS + 96, cb);
-        pass2(ca, 2);
-        tmem_wait_ld();
-        pass2(cb, 3);
+        }
         float a0, a1;
         unf2(add2(acc[0], acc[1]), a0, a1);
         l_run += a0 + a1;
@@ -620,13 +652,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (__any_sync(0xFFFFFFFFu, rescale)) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            tmem_ld32(tO + uint32_t(c) * 32, ca);
+            float o[32];
+            tmem_ld32(tO + uint32_t(c) * 32, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ca[i] *= alpha;
-            tmem_st32(tO + uint32_t(c) * 32, ca);
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(tO + uint32_t(c) * 32, o);
           }
         }
+        o_init = true;  // the P V of this tile will initialise / update O
       }
       tmem_wait_st();
       tc_fence_before();
@@ -637,31 +671,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (__all_sync(0xFFFFFFFFu, ok)) {
       tc_fence_after();
       const bool store = q_row < p.n_q;
-      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-      uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) +
-                                             (int64_t(q_row) * p.heads + head) * 128);
+      if (slot >= 0) {
+        // partial of a split item: unnormalised O, running max and sum (log2)
+        const int prow = t * 128 + r;
+        float4* po = reinterpret_cast<float4*>(p.part_o + (int64_t(slot) * 256 + prow) * 128);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float o[32];
-        if (n_iter > 0) {
-          tmem_ld32(tO + uint32_t(c) * 32, o);
-          tmem_wait_ld();
-        } else {
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          if (n_iter > 0) {
+            tmem_ld32(tO + uint32_t(c) * 32, o);
+            tmem_wait_ld();
+          }
+          if (!(n_iter > 0 && o_init && l_run > 0.f)) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0.f;
+            for (int i = 0; i < 32; ++i) o[i] = 0.f;
+          }
+          if (store) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              po[c * 8 + i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          }
         }
-        uint32_t w[16];
+        if (store) p.part_ml[int64_t(slot) * 256 + prow] = make_float2(m_run, l_run);
+      } else {
+        const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+        uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) +
+                                               (int64_t(q_row) * p.heads + head) * 128);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) w[i] = pack_bf16(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
-        if (store) {
+        for (int c = 0; c < 4; ++c) {
+          float o[32];
+          if (n_iter > 0) {
+            tmem_ld32(tO + uint32_t(c) * 32, o);
+            tmem_wait_ld();
+          }
+          if (!(n_iter > 0 && o_init && l_run > 0.f)) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            orow[c * 4 + i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            for (int i = 0; i < 32; ++i) o[i] = 0.f;
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = pack_bf16(o[2 * i] * inv_l, o[2 * i + 1] * inv_l);
+          if (store) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              orow[c * 4 + i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
         }
+        if (store && p.lse)
+          p.lse[int64_t(head) * p.n_q + q_row] =
+              l_run > 0.f ? (m_run + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
       }
-      if (store && p.lse)
-        p.lse[int64_t(head) * p.n_q + q_row] =
-            l_run > 0.f ? (m_run + __log2f(l_run)) * 0.6931471805599453f : -INFINITY;
     }
   }
 
@@ -684,9 +743,95 @@ cudaError_t launch_attention(const AttnMaps& maps, const AttnArgs& args, cudaStr
     if (e != cudaSuccess) return e;
     configured_mask |= 1 << dev;
   }
-  const unsigned grid = unsigned(args.n_pairs) * unsigned(args.heads);
+  const unsigned grid = unsigned(args.n_full) + unsigned(args.n_split) * unsigned(args.chunks);
   attn_fwd_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps.q, maps.k_cur, maps.v_cur,
                                                           maps.k_cache, maps.v_cache, args);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// merge of the key chunks of split items
+// ---------------------------------------------------------------------------
+
+// One warp per query row of a split item (32 CTAs of 8 warps per item): with
+// chunk maxima m_k and sums l_k (log2 domain) and unnormalised O_k,
+//   M = max m_k,  w_k = 2^(m_k - M),  O = sum w_k O_k / sum w_k l_k,
+//   LSE = (M + log2 sum w_k l_k) ln 2.
+// A chunk that saw no key has l_k = 0 and O_k = 0 (the attention kernel
+// stores zeros then), so it gets weight 0 and its loads need no branch.
+__global__ void __launch_bounds__(256) merge_kernel(const AttnArgs p) {
+  const int si = blockIdx.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int prow = (blockIdx.x & 31) * 8 + warp;
+  const int item = p.n_full + si;
+  const int rank = item / p.heads;
+  const int head = item - rank * p.heads;
+  const int pair = p.item_order[rank];
+  const int q_row = pair * 256 + prow;
+  if (q_row >= p.n_q) return;
+  const int64_t slot0 = int64_t(si) * p.chunks;
+  float M = -INFINITY;
+#pragma unroll 8
+  for (int k = 0; k < p.chunks; ++k) {
+    const float2 ml = p.part_ml[(slot0 + k) * 256 + prow];
+    M = ml.y > 0.f ? fmaxf(M, ml.x) : M;
+  }
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float L = 0.f;
+#pragma unroll 8
+  for (int k = 0; k < p.chunks; ++k) {
+    const float2 ml = p.part_ml[(slot0 + k) * 256 + prow];
+    const float4 v = reinterpret_cast<const float4*>(p.part_o + ((slot0 + k) * 256 + prow) * 128)[lane];
+    const float w = ml.y > 0.f ? ex2(ml.x - M) : 0.f;
+    L += w * ml.y;
+    acc.x += w * v.x;
+    acc.y += w * v.y;
+    acc.z += w * v.z;
+    acc.w += w * v.w;
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  uint2 out;
+  out.x = pack_bf16(acc.x * inv, acc.y * inv);
+  out.y = pack_bf16(acc.z * inv, acc.w * inv);
+  reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(p.o) +
+                           (int64_t(q_row) * p.heads + head) * 128)[lane] = out;
+  if (lane == 0 && p.lse)
+    p.lse[int64_t(head) * p.n_q + q_row] =
+        L > 0.f ? (M + __log2f(L)) * 0.6931471805599453f : -INFINITY;
+}
+
+cudaError_t launch_merge(const AttnArgs& args, cudaStream_t stream) {
+  if (args.n_split <= 0) return cudaSuccess;
+  merge_kernel<<<unsigned(args.n_split) * 32u, 256, 0, stream>>>(args);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// exp2 evaluators, for testing them against each other
+// ---------------------------------------------------------------------------
+
+__global__ void exp2_eval_kernel(const float* x, float* y_poly, float* y_mufu, int64_t n) {
+  const int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 2;
+  if (i + 1 < n) {
+    float a, b;
+    exp2_poly2(x[i], x[i + 1], a, b);
+    y_poly[i] = a;
+    y_poly[i + 1] = b;
+    y_mufu[i] = ex2(x[i]);
+    y_mufu[i + 1] = ex2(x[i + 1]);
+  } else if (i < n) {
+    float a, b;
+    exp2_poly2(x[i], x[i], a, b);
+    y_poly[i] = a;
+    y_mufu[i] = ex2(x[i]);
+  }
+}
+
+cudaError_t launch_exp2_eval(const float* x, float* y_poly, float* y_mufu, int64_t n,
+                             cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t threads = (n + 1) / 2;
+  exp2_eval_kernel<<<unsigned((threads + 255) / 256), 256, 0, stream>>>(x, y_poly, y_mufu, n);
   return cudaGetLastError();
 }
 

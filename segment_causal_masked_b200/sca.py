@@ -34,7 +34,9 @@ EXPORTED = (
     "sca_metadata_get_schedule", "sca_metadata_get_descriptors", "sca_metadata_upload",
     "sca_metadata_destroy", "sca_kv_cache_create", "sca_kv_cache_append",
     "sca_kv_cache_truncate", "sca_kv_cache_get", "sca_kv_cache_destroy",
-    "sca_action_causal_attn_fwd", "sca_last_error", "sca_debug_bounded_wait",
+    "sca_action_causal_attn_fwd", "sca_attn_workspace_bytes", "sca_attn_plan",
+    "sca_set_split_override",
+    "sca_last_error", "sca_debug_bounded_wait", "sca_debug_exp2",
 )
 
 
@@ -71,9 +73,14 @@ _SIGS = {
     "sca_kv_cache_truncate": [_P, _i32],
     "sca_kv_cache_get": [_P, _pi64, _pi32],
     "sca_kv_cache_destroy": [_P],
-    "sca_action_causal_attn_fwd": [_P, _P, _i32, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P],
+    "sca_action_causal_attn_fwd": [_P, _P, _i32, _P, _P, _P, _P, _P, ctypes.c_float, _P,
+                                   ctypes.c_uint64, _P, _P],
+    "sca_attn_workspace_bytes": [_P, _i32, ctypes.POINTER(ctypes.c_uint64)],
+    "sca_attn_plan": [_P, _i32, _pi32, _pi32, _pi32],
+    "sca_set_split_override": [_i32],
     "sca_last_error": [],
     "sca_debug_bounded_wait": [_P, _i64, _P],
+    "sca_debug_exp2": [_P, _P, _P, _i64, _P],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -258,13 +265,45 @@ def kv_cache_truncate(cache: KVCache, n_segments: int) -> None:
 # ---------------------------------------------------------------------------
 
 def action_causal_attn_fwd(cache: Optional[KVCache], md: Metadata, heads: int, q, k_cur, v_cur, o,
-                           lse=None, softmax_scale: float = 128 ** -0.5, dev_status=None,
+                           lse=None, softmax_scale: float = 128 ** -0.5, workspace=None,
+                           workspace_bytes: Optional[int] = None, dev_status=None,
                            stream=None) -> None:
+    """``workspace``: optional device scratch (a uint8 tensor, or an int
+    address with ``workspace_bytes``) of at least ``attn_workspace_bytes``."""
+    if workspace is not None and workspace_bytes is None:
+        workspace_bytes = int(workspace.numel() * workspace.element_size())
     _check(_lib.sca_action_causal_attn_fwd(cache.handle if cache is not None else None, md.handle,
                                            int(heads), _ptr(q), _ptr(k_cur), _ptr(v_cur), _ptr(o),
-                                           _ptr(lse), float(softmax_scale), _ptr(dev_status),
+                                           _ptr(lse), float(softmax_scale), _ptr(workspace),
+                                           int(workspace_bytes or 0), _ptr(dev_status),
                                            _stream(stream)))
+
+
+def attn_workspace_bytes(md: Metadata, heads: int) -> int:
+    """Scratch bytes the attention's split plan needs on the current device."""
+    b = ctypes.c_uint64()
+    _check(_lib.sca_attn_workspace_bytes(md.handle, int(heads), ctypes.byref(b)))
+    return int(b.value)
+
+
+def attn_plan(md: Metadata, heads: int) -> dict:
+    """The work split the next call would run (with enough workspace)."""
+    a, b, c = _i32(), _i32(), _i32()
+    _check(_lib.sca_attn_plan(md.handle, int(heads), ctypes.byref(a), ctypes.byref(b),
+                              ctypes.byref(c)))
+    return {"n_full": a.value, "n_split": b.value, "chunks": c.value}
+
+
+def set_split_override(chunks: int) -> None:
+    """0 = automatic split plan, 1 = never split, k >= 2 = split the tail into k chunks."""
+    _check(_lib.sca_set_split_override(int(chunks)))
 
 
 def debug_bounded_wait(dev_status, timeout_ns: int, stream=None) -> None:
     _check(_lib.sca_debug_bounded_wait(_ptr(dev_status), int(timeout_ns), _stream(stream)))
+
+
+def debug_exp2(x, y_poly, y_mufu, stream=None) -> None:
+    """The kernel's two exp2 evaluators on a float32 device tensor x."""
+    _check(_lib.sca_debug_exp2(_ptr(x), _ptr(y_poly), _ptr(y_mufu), int(x.numel()),
+                               _stream(stream)))

@@ -40,15 +40,21 @@ class GpuSession:
                                                   problem.textq_policy).upload()
         self.status = torch.zeros(1, dtype=torch.int32, device=self.dev)
 
-    def forward(self, q=None, k_cur=None, v_cur=None):
+    def forward(self, q=None, k_cur=None, v_cur=None, workspace=True):
+        """One attention call; with ``workspace`` the split plan's scratch is
+        passed (so the key-split tail and the merge kernel run when planned)."""
         q = self.q if q is None else q
         k_cur = self.k_cur if k_cur is None else k_cur
         v_cur = self.v_cur if v_cur is None else v_cur
         nq, h = self.p.n_query_tokens, self.p.heads
         o = torch.empty(nq, h, 128, dtype=torch.bfloat16, device=self.dev)
         lse = torch.empty(h, nq, dtype=torch.float32, device=self.dev)
+        ws = None
+        if workspace:
+            nbytes = sca.attn_workspace_bytes(self.md, h)
+            ws = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=self.dev)
         sca.action_causal_attn_fwd(self.cache if self.p.cached else None, self.md, h, q, k_cur,
-                                   v_cur, o, lse, self.p.softmax_scale, self.status)
+                                   v_cur, o, lse, self.p.softmax_scale, ws, None, self.status)
         torch.cuda.synchronize(self.dev)
         assert int(self.status.item()) == 0, f"device status {int(self.status.item())}"
         return o, lse

@@ -58,6 +58,43 @@ def test_attention_matches_oracle(p, q_scale):
     compare(o, lse, o_ref, lse_ref)
 
 
+@pytest.mark.parametrize("chunks", [2, 3, 7])
+@pytest.mark.parametrize("p", [W.small_session(), W.small_packed(seed=21, n_segments=14),
+                               W.Problem("multi-pair", SMALL[7].cached, SMALL[7].current, heads=3)],
+                         ids=lambda p: p.name if hasattr(p, "name") else str(p))
+def test_split_keys_and_merge(p, chunks):
+    """Items cut into key chunks (fp32 partials + merge kernel) match the
+    oracle and the unsplit call (up to fp32 summation order)."""
+    inputs = W.make_inputs(p, 41, 4.0)
+    s = GpuSession(p, inputs)
+    o1, l1 = s.forward(workspace=False)
+    try:
+        sca.set_split_override(chunks)
+        assert sca.attn_workspace_bytes(s.md, p.heads) > 0
+        o2, l2 = s.forward()
+    finally:
+        sca.set_split_override(0)
+    q, k, v = oracle_inputs(inputs)
+    o_ref, lse_ref = oattn.attention(orule.Layout.of(p), q, k, v, p.softmax_scale)
+    compare(o2, l2, o_ref, lse_ref)
+    assert (o1.float() - o2.float()).abs().max().item() <= 1.6e-2
+    # the FMA-pipe exp2 carries up to 7.5e-5 relative error per term, taken at
+    # different running-max offsets in the two calls: LSE may move ~1e-4
+    assert (l1 - l2).abs().max().item() <= 5e-4
+
+
+def test_split_without_workspace_falls_back():
+    p = W.small_session(heads=2)
+    s = GpuSession(p, W.make_inputs(p, 42))
+    try:
+        sca.set_split_override(3)
+        o1, l1 = s.forward(workspace=False)
+    finally:
+        sca.set_split_override(0)
+    o2, l2 = s.forward(workspace=False)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
 def test_append_is_bit_exact():
     p = W.small_session(heads=5)
     inputs = W.make_inputs(p, 32)
@@ -196,6 +233,11 @@ def test_host_side_errors():
     with pytest.raises(sca.ScaError) as e:
         sca.action_causal_attn_fwd(s.cache, s.md, 2, bad, s.k_cur, s.v_cur, o)
     assert e.value.code == sca.ERR_MISALIGNED
+    ws = torch.empty(4096, dtype=torch.uint8, device="cuda")
+    with pytest.raises(sca.ScaError) as e:
+        sca.action_causal_attn_fwd(s.cache, s.md, 2, s.q, s.k_cur, s.v_cur, o,
+                                   workspace=ws.data_ptr() + 16, workspace_bytes=1024)
+    assert e.value.code == sca.ERR_MISALIGNED
     with pytest.raises(sca.ScaError) as e:
         sca.action_causal_attn_fwd(None, s.md, 2, s.q, s.k_cur, s.v_cur, o)
     assert e.value.code == sca.ERR_MISMATCH
@@ -228,3 +270,22 @@ def test_full_size_sampled_rows(make):
     o_ref, lse_ref = oattn.attention_rows(lay, q, k, v, rows, p.softmax_scale, heads=heads)
     compare(o[rows][:, heads], lse[heads][:, rows], o_ref, lse_ref)
     assert torch.isfinite(o.float()).all()
+
+
+def test_polynomial_exp2_against_float64_and_mufu():
+    """The FMA-pipe 2^x (Cody-Waite + fitted cubic) stays within 1.5e-4
+    relative of float64 2^x on the range the kernel feeds it (x in [-126, 8]),
+    the hardware ex2.approx within 1e-6."""
+    x64 = np.concatenate([np.linspace(-126.0, 8.0, 1_000_003),
+                          np.array([-126.0, -0.5, 0.0, 0.5, 1.0, 7.999, 8.0])])
+    x = torch.from_numpy(x64.astype(np.float32)).cuda()
+    yp, ym = torch.empty_like(x), torch.empty_like(x)
+    sca.debug_exp2(x, yp, ym)
+    torch.cuda.synchronize()
+    ref = np.exp2(x.cpu().numpy().astype(np.float64))
+    rel_p = np.abs(yp.cpu().numpy().astype(np.float64) / ref - 1.0)
+    rel_m = np.abs(ym.cpu().numpy().astype(np.float64) / ref - 1.0)
+    assert rel_p.max() <= 1.5e-4, rel_p.max()
+    assert rel_m.max() <= 1e-6, rel_m.max()
+    # the minimax cubic does not interpolate 2^0 = 1: P(0) = c0, inside the bound
+    assert abs(yp[x64.size - 5].item() - 1.0) <= 7.5e-5
