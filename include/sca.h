@@ -238,6 +238,37 @@ SCA_API int sca_attn_plan(const sca_metadata* md, int32_t heads, int32_t* n_full
  * after the full waves into k chunks (a test and tuning knob). */
 SCA_API int sca_set_split_override(int32_t chunks);
 
+/* Attention forward for callers that cannot allocate device memory (no
+ * counterpart in the Hy-Nomas pages; a deployment convenience). Some callers
+ * must never call the allocator - a latency-bound inference loop (cudaMalloc
+ * can synchronise the device or fail under memory pressure), or a host
+ * runtime whose own allocator owns all device memory - and so cannot provide
+ * the workspace sca_action_causal_attn_fwd takes for its key-split partials.
+ * This variant computes exactly what sca_action_causal_attn_fwd computes with
+ * a workspace, but takes the partials from a fixed array of
+ * SCA_STATIC_WORKSPACE_BYTES that is part of the library; it allocates
+ * nothing. Arguments and results are those of sca_action_causal_attn_fwd,
+ * without the workspace.
+ *   - Limit: if the call's split plan needs more scratch than the array holds
+ *     (sca_attn_workspace_bytes), it returns SCA_ERR_CAPACITY and launches
+ *     nothing.
+ *   - Set-up: the first call on each device (with that device current) looks
+ *     up the array's device address once; make that first call before any
+ *     stream capture.
+ *   - Sharing: every call, on every stream, uses the same array, which keeps
+ *     the last call's contents. Nothing in it needs to start at zero (a call
+ *     reads only partials it wrote itself), but calls that overlap on the GPU
+ *     race: order them (one stream, or events).
+ *   - Memory: every GPU that loads the library holds the array until the
+ *     process exits. */
+#define SCA_STATIC_WORKSPACE_BYTES (32ull << 20)
+SCA_API int sca_action_causal_attn_fwd_static_ws(const sca_kv_cache* cache,
+                                                 const sca_metadata* md, int32_t heads,
+                                                 const void* q, const void* k_cur,
+                                                 const void* v_cur, void* o, float* lse,
+                                                 float softmax_scale, int32_t* dev_status,
+                                                 void* stream);
+
 /* Message of the calling thread's last failure ("" if none). */
 SCA_API const char* sca_last_error(void);
 

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsca.so")
-SOURCES = ["sca_host.cpp", "sca_kernels.cu"]
+SOURCES = ["sca_host.cpp", "sca_kernels.cu", "sca_static_ws.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -1,0 +1,78 @@
+// Attention forward for callers that cannot allocate device memory.
+//
+// Some callers must not allocate: an inference loop with a hard latency
+// budget that cannot afford the allocator (a cudaMalloc may synchronise the
+// device, and may fail under memory pressure), or a runtime that embeds this
+// library and whose own allocator owns all device memory, leaving nothing to
+// carve a workspace from. sca_action_causal_attn_fwd allocates nothing itself
+// but takes its key-split scratch from the caller. This entry point keeps
+// that scratch in one fixed array that is part of the loaded library.
+//
+// The array lives in this file as a static __device__ object of
+// SCA_STATIC_WORKSPACE_BYTES; every GPU that loads libsca holds it until the
+// process exits. Host code needs its device address (the array's name is only
+// a host-side stand-in): the first call on a device, with that device
+// current, looks it up with cudaGetSymbolAddress and remembers it.
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "sca_internal.h"
+
+namespace sca {
+
+// 32 MiB: enough for the key-split partials of the 480p long-session and
+// single-turn layouts at 16 heads on a B200 (about 29 MB at most).
+constexpr uint64_t kStaticWorkspaceBytes = SCA_STATIC_WORKSPACE_BYTES;
+
+static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_ws_mutex;
+void* g_ws_ptr[kMaxDevices] = {nullptr};
+}  // namespace
+
+// Device address of the static workspace on device `dev` (the current one).
+static int static_workspace(int dev, void** out) {
+  if (dev < 0 || dev >= kMaxDevices) return fail(SCA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_ws_mutex);
+  if (!g_ws_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (e != cudaSuccess) return check_cuda(e, "cudaGetSymbolAddress(static workspace)");
+    g_ws_ptr[dev] = p;
+  }
+  *out = g_ws_ptr[dev];
+  return SCA_OK;
+}
+
+}  // namespace sca
+
+using namespace sca;
+
+extern "C" {
+
+int sca_action_causal_attn_fwd_static_ws(const sca_kv_cache* cache, const sca_metadata* md,
+                                         int32_t heads, const void* q, const void* k_cur,
+                                         const void* v_cur, void* o, float* lse,
+                                         float softmax_scale, int32_t* dev_status,
+                                         void* stream) {
+  uint64_t need = 0;
+  if (int rc = sca_attn_workspace_bytes(md, heads, &need)) return rc;
+  if (need > kStaticWorkspaceBytes)
+    return fail(SCA_ERR_CAPACITY,
+                "this call needs %llu bytes of key-split scratch; the library's static workspace "
+                "holds %llu (use sca_action_causal_attn_fwd with a caller workspace)",
+                (unsigned long long)need, (unsigned long long)kStaticWorkspaceBytes);
+  int dev = 0;
+  if (int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
+  void* ws = nullptr;
+  if (int rc = static_workspace(dev, &ws)) return rc;
+  return sca_action_causal_attn_fwd(cache, md, heads, q, k_cur, v_cur, o, lse, softmax_scale, ws,
+                                    kStaticWorkspaceBytes, dev_status, stream);
+}
+
+}  // extern "C"

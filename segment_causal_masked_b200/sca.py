@@ -34,7 +34,8 @@ EXPORTED = (
     "sca_metadata_get_schedule", "sca_metadata_get_descriptors", "sca_metadata_upload",
     "sca_metadata_destroy", "sca_kv_cache_create", "sca_kv_cache_append",
     "sca_kv_cache_truncate", "sca_kv_cache_get", "sca_kv_cache_destroy",
-    "sca_action_causal_attn_fwd", "sca_attn_workspace_bytes", "sca_attn_plan",
+    "sca_action_causal_attn_fwd", "sca_action_causal_attn_fwd_static_ws",
+    "sca_attn_workspace_bytes", "sca_attn_plan",
     "sca_set_split_override",
     "sca_last_error", "sca_debug_bounded_wait", "sca_debug_exp2",
 )
@@ -75,6 +76,8 @@ _SIGS = {
     "sca_kv_cache_destroy": [_P],
     "sca_action_causal_attn_fwd": [_P, _P, _i32, _P, _P, _P, _P, _P, ctypes.c_float, _P,
                                    ctypes.c_uint64, _P, _P],
+    "sca_action_causal_attn_fwd_static_ws": [_P, _P, _i32, _P, _P, _P, _P, _P, ctypes.c_float,
+                                             _P, _P],
     "sca_attn_workspace_bytes": [_P, _i32, ctypes.POINTER(ctypes.c_uint64)],
     "sca_attn_plan": [_P, _i32, _pi32, _pi32, _pi32],
     "sca_set_split_override": [_i32],
@@ -277,6 +280,25 @@ def action_causal_attn_fwd(cache: Optional[KVCache], md: Metadata, heads: int, q
                                            _ptr(lse), float(softmax_scale), _ptr(workspace),
                                            int(workspace_bytes or 0), _ptr(dev_status),
                                            _stream(stream)))
+
+
+STATIC_WORKSPACE_BYTES = 32 << 20
+
+
+def action_causal_attn_fwd_static_ws(cache: Optional[KVCache], md: Metadata, heads: int, q,
+                                     k_cur, v_cur, o, lse=None,
+                                     softmax_scale: float = 128 ** -0.5, dev_status=None,
+                                     stream=None) -> None:
+    """Same result as ``action_causal_attn_fwd`` with a workspace, for callers
+    that must not allocate: the key-split scratch comes from a fixed array of
+    ``STATIC_WORKSPACE_BYTES`` inside the library (shared by all calls, so
+    calls must not overlap on the GPU). Raises ``ScaError`` with
+    ``ERR_CAPACITY`` when the call would need more scratch than that. The
+    first call on a device looks the array up and should precede any stream
+    capture."""
+    _check(_lib.sca_action_causal_attn_fwd_static_ws(
+        cache.handle if cache is not None else None, md.handle, int(heads), _ptr(q), _ptr(k_cur),
+        _ptr(v_cur), _ptr(o), _ptr(lse), float(softmax_scale), _ptr(dev_status), _stream(stream)))
 
 
 def attn_workspace_bytes(md: Metadata, heads: int) -> int:
