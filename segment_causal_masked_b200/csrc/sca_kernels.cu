@@ -18,6 +18,7 @@
 //   warps 4-7  softmax of query tile 1
 //   warp  8    TMA producer (Q once, then K_j, V_j into a 4-stage ring)
 //   warp  9    TMEM allocator and MMA issuer (one elected thread)
+//   warps 10-11 idle (they complete the control warpgroup's register split)
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,384),
 // O1 [384,512); P_t (bf16 pairs) overwrites the first 64 columns of S_t.
 // The MMA warp ping-pongs the two tiles: while softmax works on tile 0's
@@ -131,7 +132,7 @@ struct Ctl {
 // ctl->abort, writes SCA_ERR_DEVICE_TIMEOUT to *status (if any) and returns
 // false. Every pipeline wait of this file goes through here, so a broken
 // handshake ends the kernel with an error status instead of a hang.
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile Ctl* ctl,
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile Ctl* ctl,
                                           int32_t* status, unsigned long long timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
@@ -148,8 +149,9 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// Common case inline; the bounded polling loop only when the phase is not
-// complete yet (keeps the call, and its register spills, off the fast path).
+// One try first; the bounded polling loop only when the phase is not complete
+// yet. (Everything is inlined: a shared out-of-line callee would stop ptxas
+// from giving the warpgroups different register budgets.)
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile Ctl* ctl,
                                          int32_t* status, unsigned long long timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -325,6 +327,34 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// p = exp2(x * scale - m) for one row's 128 scores, summed into `acc` and
+// written as bf16 pairs over the first 64 TMEM columns of the row's S (P
+// chunk c lands in S chunk c/2, whose scores are already in registers).
+// kEvery > 0: every kEvery-th pair of exponentials is evaluated on the FMA
+// pipe (exp2_poly2, finite inputs only) instead of the MUFU.
+template <int kEvery>
+__device__ __forceinline__ void exp_pack_store(const float (&x)[128], uint64_t scale2,
+                                               uint64_t negm2, uint32_t tS, uint64_t (&acc)[2]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float x0, x1, p0, p1;
+      unf2(fma2(f2(x[32 * c + 2 * i], x[32 * c + 2 * i + 1]), scale2, negm2), x0, x1);
+      if (kEvery > 0 && (i % kEvery) == kEvery - 1) {
+        exp2_poly2(x0, x1, p0, p1);
+      } else {
+        p0 = ex2(x0);
+        p1 = ex2(x1);
+      }
+      acc[i & 1] = add2(acc[i & 1], f2(p0, p1));
+      pk[i] = pack_bf16(p0, p1);
+    }
+    tmem_st16(tS + uint32_t(c) * 16, pk);
+  }
+}
+
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -343,13 +373,22 @@ __device__ __forceinline__ bool visible(uint32_t q0, uint32_t q1, uint32_t k) {
 // ---------------------------------------------------------------------------
 
 constexpr int kStages = 4;
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;     // 3 warpgroups
+// Registers are split per warpgroup with setmaxnreg: the launch reserves
+// 384 x 168 = 64,512 (168 is the most a thread can get when three warps share
+// an SM sub-partition's 16K registers); the two softmax warpgroups grow to 224
+// (a row's 128 scores stay in registers) and the producer/MMA warpgroup
+// shrinks to 56: 2 x 128 x 224 + 128 x 56 = 64,512.
+constexpr int kRegsSoftmax = 224;
+constexpr int kRegsControl = 56;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl == kThreads * 168,
+              "the register split must add up to the launch's registers");
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kHalf = 128 * 64 * 2;  // one 128-row x 64-column bf16 box: 16 KB
 constexpr uint32_t kTile = 2 * kHalf;     // 128 x 128 bf16: 32 KB
 constexpr float kRescaleThreshold = 8.0f; // log2 units: p stays <= 2^8 between rescales
-constexpr int kPolyEvery = 4;             // 1 in 4 exponential pairs on the FMA pipe (FULL tiles)
+constexpr int kPolyEvery = 0;             // every n-th exponential pair of FULL tiles on the FMA pipe (0: none)
 
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr uint32_t kOffQ = 0;                            // Q0, Q1
@@ -426,7 +465,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kLoadWarp) {
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
+  if (warp >= 10) {
+    // warps 10-11 only complete the control warpgroup
+  } else if (warp == kLoadWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n_iter > 0) {
       const uint32_t sQ = sbase + kOffQ;
@@ -544,8 +587,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_bounded(bar(kBarDrain), 0, ctl, nullptr, p.timeout_ns);
     }
     __syncwarp();
+  }
   } else {
     // ------------------------------------------------------------ softmax
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     const int t = warp >> 2;           // query tile of the pair
     const int wq = warp & 3;           // TMEM lane quadrant
     const int r = wq * 32 + lane;      // row in the tile
@@ -619,28 +664,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
         const uint64_t negm2 = f2(neg_m, neg_m);
         uint64_t acc[2] = {0ull, 0ull};  // packed partial sums
-        // p = exp2(s * scale_log2 - m), row sum, bf16 P over the first 64
-        // columns of S (all of S is in registers already). On FULL tiles (no
-        // -inf) every kPolyEvery-th pair goes to the FMA pipe instead of the
-        // MUFU, which at d = 128 is otherwise as busy as the tensor cores.
-        const bool full_tile = cls == SCA_TILE_FULL;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float x0, x1, p0, p1;
-            unf2(fma2(f2(x[32 * c + 2 * i], x[32 * c + 2 * i + 1]), scale2, negm2), x0, x1);
-            if (kPolyEvery > 0 && (i % kPolyEvery) == kPolyEvery - 1 && full_tile) {
-              exp2_poly2(x0, x1, p0, p1);
-            } else {
-              p0 = ex2(x0);
-              p1 = ex2(x1);
-            }
-            acc[i & 1] = add2(acc[i & 1], f2(p0, p1));
-            pk[i] = pack_bf16(p0, p1);
-          }
-          tmem_st16(tS + uint32_t(c) * 16, pk);
+        // p = exp2(s * scale_log2 - m), row sum, bf16 P. FULL tiles (no -inf)
+        // may send part of the exponentials to the FMA pipe; the choice is
+        // made once per tile so the compiler keeps the two paths apart.
+        if (cls == SCA_TILE_FULL) {
+          exp_pack_store<kPolyEvery>(x, scale2, negm2, tS, acc);
+        } else {
+          exp_pack_store<0>(x, scale2, negm2, tS, acc);
         }
         float a0, a1;
         unf2(add2(acc[0], acc[1]), a0, a1);
