@@ -192,21 +192,65 @@ constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) 
                               ((128u >> 4) << 24);
 constexpr uint32_t kIdescPV = kIdescQK | (1u << 16);  // B (V) is MN-major
 
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
-                                       uint32_t acc) {
+// The eight MMAs of one 128 x 128 x 128 product (K = 8 x 16) in one asm
+// block, so the single issuing thread spends a few instructions per MMA. The
+// descriptors advance through their start-address field (bits 0..13, in
+// 16-byte units) with 32-bit adds on the low word; smem addresses stay below
+// 256 KB, so the field never carries into the next one.
+// S = Q K^T: A (Q) and B (K) K-major, 32 B per K-step inside a 64-column
+// half, 16 KB (1024 units) to the second half; D is overwritten.
+__device__ __forceinline__ void mma_qk8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                        uint32_t idesc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      "{\n\t.reg .pred pf, pt;\n\t.reg .b32 al, bl;\n\t.reg .b64 ad, bd;\n\t"
+      "setp.ne.b32 pf, 0, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\t"
+      "mov.b64 ad, {%1, %2};\n\tmov.b64 bd, {%3, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pf;\n\t"
+      "add.u32 al, %1, 2;\n\tadd.u32 bl, %3, 2;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "add.u32 al, %1, 4;\n\tadd.u32 bl, %3, 4;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "add.u32 al, %1, 6;\n\tadd.u32 bl, %3, 6;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "add.u32 al, %1, 1024;\n\tadd.u32 bl, %3, 1024;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "add.u32 al, %1, 1026;\n\tadd.u32 bl, %3, 1026;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "add.u32 al, %1, 1028;\n\tadd.u32 bl, %3, 1028;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t"
+      "add.u32 al, %1, 1030;\n\tadd.u32 bl, %3, 1030;\n\tmov.b64 ad, {al, %2};\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, pt;\n\t}"
+      ::"r"(d_tmem), "r"(uint32_t(a_desc)), "r"(uint32_t(a_desc >> 32)), "r"(uint32_t(b_desc)),
+      "r"(uint32_t(b_desc >> 32)), "r"(idesc)
       : "memory");
 }
 
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
-                                       uint32_t idesc, uint32_t acc) {
+// O (+)= P V: A = P from TMEM (8 columns per K-step of 16 keys), B = V
+// MN-major, 2048 B (128 units) per K-step. `acc` = 0 overwrites O on the
+// first K-step.
+__device__ __forceinline__ void mma_pv8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                        uint32_t idesc, uint32_t acc) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      "{\n\t.reg .pred pf, pt;\n\t.reg .b32 ta, bl;\n\t.reg .b64 bd;\n\t"
+      "setp.ne.b32 pf, %5, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\t"
+      "mov.b64 bd, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, pf;\n\t"
+      "add.u32 ta, %1, 8;\n\tadd.u32 bl, %2, 128;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %4, pt;\n\t"
+      "add.u32 ta, %1, 16;\n\tadd.u32 bl, %2, 256;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %4, pt;\n\t"
+      "add.u32 ta, %1, 24;\n\tadd.u32 bl, %2, 384;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %4, pt;\n\t"
+      "add.u32 ta, %1, 32;\n\tadd.u32 bl, %2, 512;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %4, pt;\n\t"
+      "add.u32 ta, %1, 40;\n\tadd.u32 bl, %2, 640;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %4, pt;\n\t"
+      "add.u32 ta, %1, 48;\n\tadd.u32 bl, %2, 768;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %4, pt;\n\t"
+      "add.u32 ta, %1, 56;\n\tadd.u32 bl, %2, 896;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %4, pt;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "r"(uint32_t(b_desc)), "r"(uint32_t(b_desc >> 32)), "r"(idesc),
+      "r"(acc)
       : "memory");
 }
 
@@ -342,7 +386,7 @@ __device__ __forceinline__ void exp_pack_store(const float (&x)[128], uint64_t s
     for (int i = 0; i < 16; ++i) {
       float x0, x1, p0, p1;
       unf2(fma2(f2(x[32 * c + 2 * i], x[32 * c + 2 * i + 1]), scale2, negm2), x0, x1);
-      if (kEvery > 0 && (i % kEvery) == kEvery - 1) {
+      if (kEvery > 0 && (i % (kEvery > 0 ? kEvery : 1)) == kEvery - 1) {
         exp2_poly2(x0, x1, p0, p1);
       } else {
         p0 = ex2(x0);
@@ -519,17 +563,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sQ0 = sbase + kOffQ, sQ1 = sQ0 + kTile;
       const uint32_t tS0 = tmem, tS1 = tmem + 128, tO0 = tmem + 256, tO1 = tmem + 384;
       auto issue_qk = [&](uint32_t tS, uint32_t sQ, uint32_t sK) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t off = uint32_t(k >> 2) * kHalf + uint32_t(k & 3) * 32;
-          mma_ss(tS, desc_kmajor(sQ + off), desc_kmajor(sK + off), kIdescQK, k > 0);
-        }
+        mma_qk8(tS, desc_kmajor(sQ), desc_kmajor(sK), kIdescQK);
       };
       auto issue_pv = [&](uint32_t tO, uint32_t tP, uint32_t sV, bool acc) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          mma_ts(tO, tP + uint32_t(k) * 8, desc_mnmajor(sV + uint32_t(k) * 2048), kIdescPV,
-                 (acc || k > 0) ? 1u : 0u);
+        mma_pv8(tO, tP, desc_mnmajor(sV), kIdescPV, acc ? 1u : 0u);
       };
       auto stage_of = [&](int it) { return sbase + kOffKV + uint32_t(it % kStages) * kTile; };
       auto wait_full = [&](int it) {
