@@ -38,6 +38,8 @@ WORKLOADS = {
     "480p-long-session": W.session_480p_long,
     "480p-single-turn": W.session_480p_single_turn,
     "720p-step": W.session_720p,
+    "packed-360k": W.packed_360k,
+    "tiny-packed": W.tiny_packed,
 }
 KERNEL_SOURCES = ["segment_causal_masked_b200/csrc/sca_kernels.cu",
                   "segment_causal_masked_b200/csrc/sca_internal.h"]
@@ -257,6 +259,9 @@ class Session:
             v = torch.randn(seg.n_tokens, h, 128, generator=g, device=dev).to(bf)
             self.cache.append(seg, k, v)
         self.n_prior = len(problem.cached)
+        # one current segment = an inference step (append after attention);
+        # several = a packed training-shaped forward (no cache append)
+        self.appends = len(problem.current) == 1
         self.q = torch.randn(nq, h, 128, generator=g, device=dev).to(bf)
         self.k_cur = torch.randn(nq, h, 128, generator=g, device=dev).to(bf)
         self.v_cur = torch.randn(nq, h, 128, generator=g, device=dev).to(bf)
@@ -288,9 +293,10 @@ class Session:
                                    self.workspace, None, self.status, s)
         if ev is not None:
             ev[1].record(self.stream)
-        self.cache.append(p.current[0], self.k_cur if k_cur is None else k_cur,
-                          self.v_cur if v_cur is None else v_cur, s)
-        self.cache.truncate(self.n_prior)
+        if self.appends:  # inference: the generated segment joins the cache
+            self.cache.append(p.current[0], self.k_cur if k_cur is None else k_cur,
+                              self.v_cur if v_cur is None else v_cur, s)
+            self.cache.truncate(self.n_prior)
 
 
 def run_native(args, problem):
@@ -394,7 +400,8 @@ def run_native(args, problem):
                        "cached_segments": len(problem.cached), "heads": h,
                        "head_dim": W.HEAD_DIM, "unmasked_pairs_per_head": A,
                        "effective_flop_per_step": flops,
-                       "step": "metadata build+upload, attention forward, kv_cache_append",
+                       "step": ("metadata build+upload, attention forward, kv_cache_append"
+                                if sess.appends else "metadata build+upload, attention forward"),
                        "l2": "inputs larger than L2 (cached K/V %.2f GB per tensor)"
                              % (problem.n_cache_tokens * h * 256 / 1e9),
                        "parallelism": f"replicas x{world}",
@@ -406,7 +413,7 @@ def run_native(args, problem):
                          "peak_source": f"{peaks['source']} bf16 dense (burst)"},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": bytes_in,
                     "d2h_bytes_per_step": bytes_out, "ms_per_step": e2e_ms / args.steps},
-            "gpu_launches": (2 + (1 if sess.splits else 0)) * args.steps,
+            "gpu_launches": (1 + int(sess.appends) + int(sess.splits)) * args.steps,
             "clocks": clock_info,
         }
         if not args.no_cpu_baseline:
@@ -430,7 +437,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="480p-long-session")
     ap.add_argument("--oracle-rows", type=int, default=384,
                     help="query rows per step of the reference arm")
-    ap.add_argument("--baseline-rows", type=int, default=1536,
+    ap.add_argument("--baseline-rows", type=int, default=6144,
                     help="query rows of the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -289,3 +289,20 @@ def test_polynomial_exp2_against_float64_and_mufu():
     assert rel_m.max() <= 1e-6, rel_m.max()
     # the minimax cubic does not interpolate 2^0 = 1: P(0) = c0, inside the bound
     assert abs(yp[x64.size - 5].item() - 1.0) <= 7.5e-5
+
+
+@pytest.mark.slow
+def test_packed_360k_sampled_rows():
+    """The packed training-shaped forward (~360k tokens, every token a query):
+    sampled rows against the oracle, row by row."""
+    p = W.packed_360k()
+    inputs = W.make_inputs(p, 43)
+    s = GpuSession(p, inputs)
+    o, lse = s.forward()
+    rows = W.sample_rows(p.n_query_tokens, 40, seed=2)
+    heads = [3, 12]
+    q, k, v = oracle_inputs(inputs)
+    lay = orule.Layout.of(p)
+    o_ref, lse_ref = oattn.attention_rows(lay, q, k, v, rows, p.softmax_scale, heads=heads)
+    compare(o[rows][:, heads], lse[heads][:, rows], o_ref, lse_ref)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
