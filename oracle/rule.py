@@ -27,6 +27,17 @@ Readings where the pages are silent (each is listed in the design notes):
   own segment and, like video queries, the video and heads of earlier
   segments.
 * Windows are half-open latent-frame ranges local to the segment.
+
+Two options for single-GPU inference, named on the pages without their rules
+([picx] "Inference": sliding-window attention and sparse attention keeping a
+quarter of the video blocks), read here as:
+
+* ``history`` W >= 0: a query of segment s sees earlier segments s-W .. s-1
+  only (its own segment as always); W < 0 keeps the whole history.
+* ``keep_blocks`` [query tiles, key tiles]: a False entry drops, for the
+  queries of that 128-query tile, every key of that 128-key tile when the key
+  tile holds video tokens only ("a video block"); tiles with any text key are
+  always kept. Tiles are those of the schedule (schedule.py).
 """
 from __future__ import annotations
 
@@ -114,7 +125,7 @@ def query_runs(cached: Sequence, current: Sequence) -> List[QueryRun]:
 
 
 def visible_key_ranges(all_spans: Sequence[Span], run: QueryRun,
-                       policy: int = OWN_TAIL) -> List[Tuple[int, int]]:
+                       policy: int = OWN_TAIL, history: int = -1) -> List[Tuple[int, int]]:
     """The key ranges a query of ``run`` may attend to."""
     text_query = run.kind != VIDEO
     sees_past = (not text_query) or policy == FULL_SEGMENT
@@ -123,7 +134,8 @@ def visible_key_ranges(all_spans: Sequence[Span], run: QueryRun,
         if sp.segment > run.segment:
             continue                                   # never a later segment
         if sp.segment < run.segment:
-            if sees_past:
+            in_window = history < 0 or run.segment - sp.segment <= history
+            if sees_past and in_window:
                 out += [sp.video, sp.head]             # past video + head; past tails never
             continue
         out += [sp.video, sp.head]                     # own segment: bidirectional
@@ -139,39 +151,63 @@ def visible_key_ranges(all_spans: Sequence[Span], run: QueryRun,
 class Layout:
     """Key spans and query runs of one call (cached segments, then current)."""
 
-    def __init__(self, cached: Sequence, current: Sequence, policy: int = OWN_TAIL):
+    def __init__(self, cached: Sequence, current: Sequence, policy: int = OWN_TAIL,
+                 history: int = -1, keep_blocks=None):
         self.cached = tuple(cached)
         self.current = tuple(current)
         self.policy = policy
+        self.history = history
         self.spans = spans(list(cached) + list(current))
         self.runs = query_runs(cached, current)
         self.n_keys = self.spans[-1].stop if self.spans else 0
         self.n_cache = self.spans[len(cached) - 1].stop if cached else 0
         self.n_queries = self.runs[-1].stop if self.runs else 0
         self._run_starts = np.array([r.start for r in self.runs], dtype=np.int64)
-        self._row_cache: Dict[int, np.ndarray] = {}
+        self._row_cache: Dict[Tuple[int, int], np.ndarray] = {}
+        self.keep_blocks = None if keep_blocks is None else np.asarray(keep_blocks, dtype=bool)
+        if self.keep_blocks is not None:
+            # key tiles of each source (128 keys, cache first), and which hold video only
+            is_video = np.zeros(self.n_keys, dtype=bool)
+            for sp in self.spans:
+                is_video[sp.video[0]:sp.video[1]] = True
+            self._tiles = []
+            for base, n in ((0, self.n_cache), (self.n_cache, self.n_queries)):
+                for t0 in range(0, n, 128):
+                    a, b = base + t0, base + min(n, t0 + 128)
+                    self._tiles.append((a, b, bool(is_video[a:b].all())))
+            n_qt = (self.n_queries + 127) // 128
+            if self.keep_blocks.shape != (n_qt, len(self._tiles)):
+                raise ValueError("keep_blocks must be [query tiles, key tiles]")
 
     @classmethod
     def of(cls, problem) -> "Layout":
-        return cls(problem.cached, problem.current, problem.textq_policy)
+        return cls(problem.cached, problem.current, problem.textq_policy,
+                   getattr(problem, "history_segments", -1), getattr(problem, "keep_blocks", None))
 
     def run_of(self, query: int) -> QueryRun:
         i = int(np.searchsorted(self._run_starts, query, side="right")) - 1
         return self.runs[i]
 
     def ranges(self, query: int) -> List[Tuple[int, int]]:
-        return visible_key_ranges(self.spans, self.run_of(query), self.policy)
+        """Visible key ranges of ``query`` (before any dropped video block)."""
+        return visible_key_ranges(self.spans, self.run_of(query), self.policy, self.history)
 
     def mask_row(self, query: int) -> np.ndarray:
-        """Boolean row of the explicit mask (shared by the queries of a run)."""
+        """Boolean row of the explicit mask."""
         run = self.run_of(query)
-        row = self._row_cache.get(run.start)
+        qt = query // 128 if self.keep_blocks is not None else -1
+        key = (run.start, qt)
+        row = self._row_cache.get(key)
         if row is None:
             row = np.zeros(self.n_keys, dtype=bool)
-            for a, b in visible_key_ranges(self.spans, run, self.policy):
+            for a, b in visible_key_ranges(self.spans, run, self.policy, self.history):
                 row[a:b] = True
+            if self.keep_blocks is not None:
+                for kt, (a, b, video_only) in enumerate(self._tiles):
+                    if video_only and not self.keep_blocks[qt, kt]:
+                        row[a:b] = False             # a dropped video block
             if len(self._row_cache) < max(16, (1 << 28) // max(1, self.n_keys)):
-                self._row_cache[run.start] = row
+                self._row_cache[key] = row
         return row
 
     def mask_rows(self, rows: Sequence[int]) -> np.ndarray:
@@ -188,9 +224,13 @@ class Layout:
     def unmasked_pairs(self) -> int:
         """A of Eq. 6 ([picx] Training Infrastructure; [xyznot] "Dağıtık
         Paketleme FLOP Tahmini"): the number of (query, key) pairs whose mask
-        entry is not -inf, summed run by run from the visible ranges."""
+        entry is not -inf, summed run by run from the visible ranges (row by
+        row from the explicit mask when video blocks are dropped)."""
+        if self.keep_blocks is not None:
+            return int(sum(int(self.mask_row(q).sum()) for q in range(self.n_queries)))
         total = 0
         for run in self.runs:
-            seen = sum(b - a for a, b in visible_key_ranges(self.spans, run, self.policy))
+            seen = sum(b - a for a, b in
+                       visible_key_ranges(self.spans, run, self.policy, self.history))
             total += (run.stop - run.start) * seen
         return total

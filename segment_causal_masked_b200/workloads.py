@@ -61,6 +61,8 @@ class Problem:
     current: Tuple[Segment, ...]
     heads: int = 16
     textq_policy: int = TEXTQ_OWN_TAIL
+    history_segments: int = -1          # sliding window over earlier segments (-1: all)
+    keep_blocks: object = None          # [query tiles, key tiles] bools, or None
 
     @property
     def softmax_scale(self) -> float:
@@ -203,6 +205,30 @@ def small_packed(heads: int = 3, seed: int = 12, n_segments: int = 6) -> Problem
             acts.append(Action(int(rng.integers(1, 20)), b, e))
         segs.append(Segment(f, g, int(rng.integers(0, 40)), tuple(acts)))
     return Problem("small-packed", (), tuple(segs), heads=heads)
+
+
+def with_history(problem: Problem, segments: int) -> Problem:
+    """The same call with a sliding window of ``segments`` earlier segments."""
+    return dataclasses.replace(problem, name=f"{problem.name}-window{segments}",
+                               history_segments=segments)
+
+
+def n_query_tiles(problem: Problem) -> int:
+    return (problem.n_query_tokens + 127) // 128
+
+
+def n_key_tiles(problem: Problem) -> int:
+    return (problem.n_cache_tokens + 127) // 128 + (problem.n_query_tokens + 127) // 128
+
+
+def with_random_blocks(problem: Problem, keep: float, seed: int) -> Problem:
+    """The same call keeping a seeded random fraction ``keep`` of each query
+    tile's key tiles (only video-only key tiles can be dropped; the others
+    are kept whatever the draw)."""
+    rng = np.random.default_rng(seed)
+    mask = rng.random((n_query_tiles(problem), n_key_tiles(problem))) < keep
+    return dataclasses.replace(problem, name=f"{problem.name}-blocks{int(round(100 * keep))}",
+                               keep_blocks=mask)
 
 
 CONFIGS = {

@@ -166,13 +166,14 @@ def _brute_mask(problem):
     keys = _token_table(segs)
     queries = keys[problem.n_cache_tokens:]
     full = problem.textq_policy == W.TEXTQ_FULL_SEGMENT
+    hist = problem.history_segments
     m = np.zeros((len(queries), len(keys)), dtype=bool)
     for i, (qs, qk, qf, qa) in enumerate(queries):
         for j, (ks, kk, kf, ka) in enumerate(keys):
             if ks > qs:
                 ok = False
             elif ks < qs:
-                ok = kk != "t" and (qk == "v" or full)
+                ok = kk != "t" and (qk == "v" or full) and (hist < 0 or qs - ks <= hist)
             elif kk != "t":
                 ok = True
             elif qk == "v":
@@ -181,6 +182,16 @@ def _brute_mask(problem):
             else:
                 ok = full or (qk == "t" and qa == ka)
             m[i, j] = ok
+    if problem.keep_blocks is not None:                 # drop video-only key tiles
+        nc = problem.n_cache_tokens
+        starts = list(range(0, nc, 128)) + [nc + u for u in range(0, len(queries), 128)]
+        ends = [min(nc, a + 128) for a in range(0, nc, 128)] + \
+               [nc + min(len(queries), u + 128) for u in range(0, len(queries), 128)]
+        for kt, (a, b) in enumerate(zip(starts, ends)):
+            if all(keys[j][1] == "v" for j in range(a, b)):
+                for i in range(len(queries)):
+                    if not problem.keep_blocks[i // 128, kt]:
+                        m[i, a:b] = False
     return m
 
 
@@ -199,6 +210,47 @@ def test_mask_matches_brute_force(problem):
     m = lay.mask()
     assert np.array_equal(m, _brute_mask(problem))
     assert lay.unmasked_pairs() == int(m.sum())
+
+
+def _window_and_blocks_problems():
+    sess = W.small_session(heads=1)
+    long_sess = W.Problem("long-small", tuple(W.small_packed(seed=5, n_segments=7).current),
+                          (W.Segment(3, 60, 9, (W.Action(4, 0, 2), W.Action(6, 1, 3))),), heads=1)
+    return [
+        W.with_history(sess, 0), W.with_history(sess, 1), W.with_history(sess, 2),
+        W.with_history(long_sess, 3),
+        W.with_history(W.small_packed(seed=21, n_segments=14), 2),
+        W.with_random_blocks(long_sess, 0.25, 7),
+        W.with_random_blocks(W.with_history(long_sess, 4), 0.5, 8),
+        W.with_random_blocks(W.small_packed(seed=21, n_segments=14), 0.3, 9),
+    ]
+
+
+@pytest.mark.parametrize("p", _window_and_blocks_problems(), ids=lambda p: p.name)
+def test_window_and_dropped_blocks_match_brute_force(p):
+    lay = orule.Layout.of(p)
+    m = lay.mask()
+    assert np.array_equal(m, _brute_mask(p))
+    assert lay.unmasked_pairs() == int(m.sum())
+
+
+def test_window_closed_form_480p():
+    """Window of 4 segments over the 12-segment cache: a video query sees 4
+    cached segments' video + head (4 x 12,218) plus its own 12,250; text
+    queries are unaffected (they never look back)."""
+    s = W.seg_480p()
+    lay = orule.Layout((s,) * 12, (s,), history=4)
+    expect = 12_090 * (4 * 12_218 + 12_250) + 128 * 12_218 + 128 * 12_250
+    assert lay.unmasked_pairs() == expect == 742_096_884   # 12,090 x 61,122 + 1,563,904 + 1,568,000
+
+
+def test_window_and_blocks_degenerate_cases():
+    p = W.small_session(heads=1)
+    full = orule.Layout.of(p).mask()
+    assert np.array_equal(orule.Layout.of(W.with_history(p, 99)).mask(), full)
+    keep_all = np.ones((W.n_query_tiles(p), W.n_key_tiles(p)), bool)
+    import dataclasses
+    assert np.array_equal(orule.Layout.of(dataclasses.replace(p, keep_blocks=keep_all)).mask(), full)
 
 
 def test_schedule_matches_brute_force_tiles():
