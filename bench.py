@@ -40,6 +40,10 @@ WORKLOADS = {
     "720p-step": W.session_720p,
     "packed-360k": W.packed_360k,
     "tiny-packed": W.tiny_packed,
+    # inference options (sliding window of 4 earlier segments; a quarter of
+    # the video blocks kept, drawn at random with a fixed seed)
+    "480p-long-session-window4": lambda: W.with_history(W.session_480p_long(), 4),
+    "480p-long-session-blocks25": lambda: W.with_random_blocks(W.session_480p_long(), 0.25, 25),
 }
 KERNEL_SOURCES = ["segment_causal_masked_b200/csrc/sca_kernels.cu",
                   "segment_causal_masked_b200/csrc/sca_internal.h"]
@@ -268,8 +272,7 @@ class Session:
         self.o = torch.empty(nq, h, 128, dtype=bf, device=dev)
         self.lse = torch.empty(h, nq, dtype=torch.float32, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
-        self.md = sca.Metadata()
-        self.md.build(problem.cached, problem.current, problem.textq_policy)
+        self.md = sca.build_for(problem)
         ws_bytes = sca.attn_workspace_bytes(self.md, h)
         self.splits = ws_bytes > 0
         self.plan = sca.attn_plan(self.md, h)
@@ -282,7 +285,7 @@ class Session:
         attention kernel."""
         sca, p = self.sca, self.p
         s = self.stream.cuda_stream
-        self.md.build(p.cached, p.current, p.textq_policy)
+        sca.build_for(p, self.md)
         self.md.upload(s)
         if ev is not None:
             ev[0].record(self.stream)
@@ -323,7 +326,7 @@ def run_native(args, problem):
 
     sess = Session(problem, seed=1000 * 2 + rank)
     from segment_causal_masked_b200 import sca
-    sca_md = sca.build_segment_mask_metadata(problem.cached, problem.current, problem.textq_policy)
+    sca_md = sca.build_for(problem)
     counts = sca_md.counts()
     A = counts["unmasked_pairs"]
     flops = effective_flops(problem, A)

@@ -140,6 +140,34 @@ SCA_API int sca_build_segment_mask_metadata(sca_metadata* md,
                                     const sca_segment* current, int32_t n_current,
                                     int32_t textq_policy);
 
+/* Options of the mask (all optional; zero-initialise and set what you need).
+ * The inference path of the Hy-Nomas report names sliding-window attention
+ * and sparse attention that keeps a quarter of the video blocks (picx.dev
+ * summary, "Inference") without their rules; this library reads them as:
+ *   history_segments W >= 0: a query of segment s sees earlier segments
+ *     s-W .. s-1 only (its own segment as always); -1 (or any negative) keeps
+ *     the whole history. 0 is a valid window (no earlier segment).
+ *   keep_blocks: NULL keeps everything; else n_q_tiles * n_kv_tiles bytes,
+ *     row-major [query tile][key tile] (tiles as in the schedule; get the
+ *     counts from a build without it): a 0 entry drops, for that query tile,
+ *     the whole key tile when it holds video tokens only ("a video block").
+ *     Key tiles with any text key are kept whatever the entry. Dropped
+ *     blocks leave the schedule and the unmasked-pair count. */
+typedef struct sca_mask_options {
+  int32_t textq_policy;
+  int32_t history_segments;
+  const uint8_t* keep_blocks;
+  int64_t keep_blocks_len;
+} sca_mask_options;
+
+/* sca_build_segment_mask_metadata with options (opt may be NULL: defaults,
+ * i.e. SCA_TEXTQ_OWN_TAIL, whole history, every block).
+ * SCA_ERR_INVALID_ARG if keep_blocks_len does not match the layout's tiles. */
+SCA_API int sca_build_segment_mask_metadata_ex(sca_metadata* md,
+                                               const sca_segment* cached, int32_t n_cached,
+                                               const sca_segment* current, int32_t n_current,
+                                               const sca_mask_options* opt);
+
 /* Sizes and totals of the last build. Any output pointer may be NULL.
  *   unmasked_pairs: A (pairs whose mask entry is not -inf), per head;
  *   n_queries / n_cache_keys: token counts; n_q_tiles, n_kv_tiles: tiles;

@@ -90,13 +90,15 @@ uint32_t key_descriptor(const SegLayout& s, uint32_t seg, int64_t t) {
 }
 
 // The pair predicate: may a query described by (q0, q1) see key `k`?
-static inline bool visible(uint32_t q0, uint32_t q1, uint32_t k) {
+// `window`: how many earlier segments a query may see (65535: all).
+static inline bool visible(uint32_t q0, uint32_t q1, uint32_t k, uint32_t window) {
   if (!(q0 & SCA_QDESC_VALID)) return false;
   const uint32_t qs = q0 & SCA_DESC_SEG_MASK, ks = k & SCA_DESC_SEG_MASK;
   if (ks == qs)  // own segment: everything but the tails outside the query's set
     return !(k & SCA_DESC_TAIL) || ((q1 >> ((k >> SCA_DESC_ACTION_SHIFT) & 31u)) & 1u);
-  // earlier segment: its live (video, head) keys, if the query looks back
-  return ks < qs && (q0 & SCA_QDESC_SEES_PAST) && (k & SCA_DESC_ALIVE);
+  // earlier segment inside the window: its live (video, head) keys, if the
+  // query looks back
+  return ks < qs && qs - ks <= window && (q0 & SCA_QDESC_SEES_PAST) && (k & SCA_DESC_ALIVE);
 }
 
 namespace {
@@ -107,28 +109,39 @@ struct TileSummary {
   bool oob = false;          // fewer than 128 existing rows
   bool all_flag = true;      // every row sees the past / every key alive
   bool any_flag = false;
+  bool video_only = true;    // keys: no head or tail key in the tile
   std::vector<uint64_t> vals;  // distinct descriptors (query: q0 | q1 << 32)
+  std::vector<int32_t> count;  // how many rows / keys carry each
   void add(uint64_t v, uint32_t seg, bool flag) {
     seg_min = std::min(seg_min, seg);
     seg_max = std::max(seg_max, seg);
     all_flag &= flag;
     any_flag |= flag;
-    if (std::find(vals.begin(), vals.end(), v) == vals.end()) vals.push_back(v);
+    auto it = std::find(vals.begin(), vals.end(), v);
+    if (it == vals.end()) {
+      vals.push_back(v);
+      count.push_back(1);
+    } else {
+      ++count[size_t(it - vals.begin())];
+    }
   }
 };
 
-uint8_t classify(const TileSummary& q, const TileSummary& k) {
+uint8_t classify(const TileSummary& q, const TileSummary& k, uint32_t window) {
   if (q.vals.empty() || k.vals.empty()) return SCA_TILE_EMPTY;
   if (k.seg_min > q.seg_max) return SCA_TILE_EMPTY;   // only later segments
   if (k.seg_max < q.seg_min) {                          // only earlier segments
-    if (!q.any_flag || !k.any_flag) return SCA_TILE_EMPTY;
-    if (q.all_flag && k.all_flag && !q.oob && !k.oob) return SCA_TILE_FULL;
-    return SCA_TILE_PARTIAL;
+    if (q.seg_min - k.seg_max > window) return SCA_TILE_EMPTY;  // all outside the window
+    if (q.seg_max - k.seg_min <= window) {                      // all inside it
+      if (!q.any_flag || !k.any_flag) return SCA_TILE_EMPTY;
+      if (q.all_flag && k.all_flag && !q.oob && !k.oob) return SCA_TILE_FULL;
+      return SCA_TILE_PARTIAL;
+    }
   }
   bool any = false, all = !q.oob && !k.oob;
   for (uint64_t qv : q.vals)
     for (uint64_t kv : k.vals) {
-      const bool v = visible(uint32_t(qv), uint32_t(qv >> 32), uint32_t(kv));
+      const bool v = visible(uint32_t(qv), uint32_t(qv >> 32), uint32_t(kv), window);
       any |= v;
       all &= v;
     }
@@ -165,6 +178,20 @@ void sca_metadata_destroy(sca_metadata* md) {
 int sca_build_segment_mask_metadata(sca_metadata* md, const sca_segment* cached,
                                     int32_t n_cached, const sca_segment* current,
                                     int32_t n_current, int32_t policy) {
+  sca_mask_options opt;
+  memset(&opt, 0, sizeof(opt));
+  opt.textq_policy = policy;
+  opt.history_segments = -1;
+  return sca_build_segment_mask_metadata_ex(md, cached, n_cached, current, n_current, &opt);
+}
+
+int sca_build_segment_mask_metadata_ex(sca_metadata* md, const sca_segment* cached,
+                                       int32_t n_cached, const sca_segment* current,
+                                       int32_t n_current, const sca_mask_options* opt) {
+  const int32_t policy = opt ? opt->textq_policy : SCA_TEXTQ_OWN_TAIL;
+  const uint32_t window = (opt && opt->history_segments >= 0)
+                              ? uint32_t(std::min(opt->history_segments, 65535)) : 65535u;
+  const uint8_t* keep = opt ? opt->keep_blocks : nullptr;
   if (!md) return fail(SCA_ERR_INVALID_ARG, "null metadata handle");
   if (n_cached < 0 || n_current < 1)
     return fail(SCA_ERR_INVALID_ARG, "need n_cached >= 0 and n_current >= 1");
@@ -216,7 +243,9 @@ int sca_build_segment_mask_metadata(sca_metadata* md, const sca_segment* cached,
       const SegLayout& S = segs[g];
       const int64_t own_live = S.n_video() + S.h;
       auto emit = [&](int64_t count, uint32_t w0, uint32_t w1) {
-        int64_t seen = own_live + ((w0 & SCA_QDESC_SEES_PAST) ? alive_before[g] : 0);
+        const int64_t first = std::max<int64_t>(0, int64_t(g) - int64_t(window));  // oldest visible
+        int64_t seen = own_live + ((w0 & SCA_QDESC_SEES_PAST)
+                                       ? alive_before[g] - alive_before[size_t(first)] : 0);
         for (int a = 0; a < S.n_act; ++a)
           if ((w1 >> a) & 1u) seen += S.len[a];
         A += count * seen;
@@ -249,40 +278,23 @@ int sca_build_segment_mask_metadata(sca_metadata* md, const sca_segment* cached,
   }
   qs[size_t(n_qt - 1)].oob = (n_q % SCA_TILE) != 0;
   auto add_keys = [&](const std::vector<uint32_t>& d, int64_t n, int64_t tile0) {
-    for (int64_t i = 0; i < n; ++i)
-      ks[size_t(tile0 + i / SCA_TILE)].add(d[size_t(i)], d[size_t(i)] & SCA_DESC_SEG_MASK,
-                                           (d[size_t(i)] & SCA_DESC_ALIVE) != 0);
+    for (int64_t i = 0; i < n; ++i) {
+      TileSummary& K = ks[size_t(tile0 + i / SCA_TILE)];
+      K.add(d[size_t(i)], d[size_t(i)] & SCA_DESC_SEG_MASK, (d[size_t(i)] & SCA_DESC_ALIVE) != 0);
+      if (d[size_t(i)] & (SCA_DESC_HEAD | SCA_DESC_TAIL)) K.video_only = false;
+    }
     if (n % SCA_TILE) ks[size_t(tile0 + n / SCA_TILE)].oob = true;
   };
   add_keys(kdesc_cache, n_cache, 0);
   add_keys(kdesc_cur, n_q, n_ct);
-
-  // --- classification and CSR ---------------------------------------------
-  std::vector<int32_t> row_ptr(size_t(n_qt) + 1, 0), kv_tile;
-  std::vector<uint8_t> flag;
-  int64_t n_full = 0, n_partial = 0;
-  kv_tile.reserve(size_t(n_qt) * 64);
-  flag.reserve(size_t(n_qt) * 64);
-  for (int qt = 0; qt < n_qt; ++qt) {
-    const TileSummary& Q = qs[size_t(qt)];
-    for (int64_t kt = 0; kt < n_ct + n_ut; ++kt) {
-      const TileSummary& K = ks[size_t(kt)];
-      if (kt < n_ct && K.seg_min > Q.seg_max) { kt = n_ct - 1; continue; }  // rest of cache is later
-      if (kt >= n_ct && K.seg_min > Q.seg_max) break;
-      const uint8_t c = classify(Q, K);
-      if (c == SCA_TILE_EMPTY) continue;
-      kv_tile.push_back(int32_t(kt));
-      flag.push_back(c);
-      (c == SCA_TILE_FULL ? n_full : n_partial) += 1;
-    }
-    row_ptr[size_t(qt) + 1] = int32_t(kv_tile.size());
-    if (kv_tile.size() > size_t(INT32_MAX) - 4096)
-      return fail(SCA_ERR_UNSUPPORTED, "schedule larger than 2^31 entries");
-  }
+  const int64_t n_kt = n_ct + n_ut;
+  if (keep && (opt->keep_blocks_len != int64_t(n_qt) * n_kt))
+    return fail(SCA_ERR_INVALID_ARG, "keep_blocks has %lld entries, the layout has %d x %lld tiles",
+                (long long)opt->keep_blocks_len, n_qt, (long long)n_kt);
 
   // --- runs of equal descriptors inside each key tile (for the kernel's
-  // per-row visibility masks on PARTIAL tiles) ---------------------------
-  std::vector<int32_t> run_ptr(size_t(n_ct + n_ut) + 1, 0);
+  // per-row visibility masks on PARTIAL tiles, and to count dropped pairs) --
+  std::vector<int32_t> run_ptr(size_t(n_kt) + 1, 0);
   std::vector<uint32_t> runs;
   auto add_runs = [&](const std::vector<uint32_t>& d, int64_t n, int64_t tile0) {
     for (int64_t t = 0; t * SCA_TILE < n; ++t) {
@@ -300,6 +312,43 @@ int sca_build_segment_mask_metadata(sca_metadata* md, const sca_segment* cached,
   };
   add_runs(kdesc_cache, n_cache, 0);
   add_runs(kdesc_cur, n_q, n_ct);
+  // visible (query, key) pairs of one tile pair, for blocks that are dropped
+  auto block_pairs = [&](const TileSummary& Q, int64_t kt) {
+    int64_t n = 0;
+    for (size_t a = 0; a < Q.vals.size(); ++a)
+      for (int32_t r = run_ptr[size_t(kt)]; r < run_ptr[size_t(kt) + 1]; ++r)
+        if (visible(uint32_t(Q.vals[a]), uint32_t(Q.vals[a] >> 32), runs[size_t(2 * r + 1)], window))
+          n += int64_t(Q.count[a]) * int64_t((runs[size_t(2 * r)] >> 8) & 255u);
+    return n;
+  };
+
+  // --- classification and CSR ---------------------------------------------
+  std::vector<int32_t> row_ptr(size_t(n_qt) + 1, 0), kv_tile;
+  std::vector<uint8_t> flag;
+  int64_t n_full = 0, n_partial = 0, n_dropped = 0;
+  kv_tile.reserve(size_t(n_qt) * 64);
+  flag.reserve(size_t(n_qt) * 64);
+  for (int qt = 0; qt < n_qt; ++qt) {
+    const TileSummary& Q = qs[size_t(qt)];
+    for (int64_t kt = 0; kt < n_ct + n_ut; ++kt) {
+      const TileSummary& K = ks[size_t(kt)];
+      if (kt < n_ct && K.seg_min > Q.seg_max) { kt = n_ct - 1; continue; }  // rest of cache is later
+      if (kt >= n_ct && K.seg_min > Q.seg_max) break;
+      const uint8_t c = classify(Q, K, window);
+      if (c == SCA_TILE_EMPTY) continue;
+      if (keep && !keep[size_t(qt) * size_t(n_kt) + size_t(kt)] && K.video_only) {
+        A -= block_pairs(Q, kt);  // a dropped video block
+        ++n_dropped;
+        continue;
+      }
+      kv_tile.push_back(int32_t(kt));
+      flag.push_back(c);
+      (c == SCA_TILE_FULL ? n_full : n_partial) += 1;
+    }
+    row_ptr[size_t(qt) + 1] = int32_t(kv_tile.size());
+    if (kv_tile.size() > size_t(INT32_MAX) - 4096)
+      return fail(SCA_ERR_UNSUPPORTED, "schedule larger than 2^31 entries");
+  }
 
   // --- kernel work list: query-tile pairs, union of their key tiles --------
   const int n_pairs = (n_qt + 1) / 2;
@@ -344,6 +393,8 @@ int sca_build_segment_mask_metadata(sca_metadata* md, const sca_segment* cached,
   md->n_cached = n_cached;
   md->n_current = n_current;
   md->policy = policy;
+  md->history = int32_t(window);
+  md->n_dropped = n_dropped;
   md->segs.swap(segs);
   md->n_cache = n_cache;
   md->n_q = n_q;
@@ -773,6 +824,7 @@ int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md
   a.n_cache_tiles = md->n_cache_tiles;
   a.heads = heads;
   a.n_pairs = md->n_pairs;
+  a.history = md->history;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
   a.timeout_ns = 2000000000ull;
   const bool split = md->plan_chunks > 1 && workspace && workspace_bytes >= md->plan_ws;

@@ -81,6 +81,7 @@ struct AttnArgs {
   int32_t n_cache_tiles;
   int32_t heads;
   int32_t n_pairs;
+  int32_t history;             // earlier segments a query may see (65535: all)
   float scale_log2;            // softmax_scale * log2(e)
   unsigned long long timeout_ns;
 };
@@ -129,6 +130,8 @@ size_t attention_smem_bytes();
 struct sca_metadata {
   bool built = false;
   int32_t n_cached = 0, n_current = 0, policy = 0;
+  int32_t history = 65535;            // window over earlier segments (65535: all)
+  int64_t n_dropped = 0;              // video blocks dropped by keep_blocks
   std::vector<sca::SegLayout> segs;   // cached then current
   int64_t n_cache = 0;                // cached keys
   int64_t n_q = 0;                    // queries = current keys

@@ -403,12 +403,14 @@ __device__ __forceinline__ void named_sync(uint32_t id, uint32_t threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// The pair predicate on descriptor words (layout documented in sca.h).
-__device__ __forceinline__ bool visible(uint32_t q0, uint32_t q1, uint32_t k) {
+// The pair predicate on descriptor words (layout documented in sca.h);
+// `window` = how many earlier segments a query may see (65535: all).
+__device__ __forceinline__ bool visible(uint32_t q0, uint32_t q1, uint32_t k, uint32_t window) {
   const uint32_t qs = q0 & SCA_DESC_SEG_MASK, ks = k & SCA_DESC_SEG_MASK;
   const bool own = (ks == qs) && (!(k & SCA_DESC_TAIL) ||
                                   ((q1 >> ((k >> SCA_DESC_ACTION_SHIFT) & 31u)) & 1u));
-  const bool past = (ks < qs) && (q0 & SCA_QDESC_SEES_PAST) && (k & SCA_DESC_ALIVE);
+  const bool past = (ks < qs) && (qs - ks <= window) && (q0 & SCA_QDESC_SEES_PAST) &&
+                    (k & SCA_DESC_ALIVE);
   return (q0 & SCA_QDESC_VALID) && (own || past);
 }
 
@@ -654,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r0 = p.run_ptr[tile], r1 = p.run_ptr[tile + 1];
         for (int i = r0; i < r1; ++i) {
           const uint2 run = p.runs[i];
-          if (!visible(qd.x, qd.y, run.y)) continue;
+          if (!visible(qd.x, qd.y, run.y, uint32_t(p.history))) continue;
           const int a = int(run.x & 255u), b = a + int((run.x >> 8) & 255u);
 #pragma unroll
           for (int w = 0; w < 4; ++w) {

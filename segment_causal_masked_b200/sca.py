@@ -30,7 +30,8 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED = 0, -1, -2, -3
 ERR_CAPACITY, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_MISMATCH = -4, -5, -6, -7
 
 EXPORTED = (
-    "sca_metadata_create", "sca_build_segment_mask_metadata", "sca_metadata_get_counts",
+    "sca_metadata_create", "sca_build_segment_mask_metadata",
+    "sca_build_segment_mask_metadata_ex", "sca_metadata_get_counts",
     "sca_metadata_get_schedule", "sca_metadata_get_descriptors", "sca_metadata_upload",
     "sca_metadata_destroy", "sca_kv_cache_create", "sca_kv_cache_append",
     "sca_kv_cache_truncate", "sca_kv_cache_get", "sca_kv_cache_destroy",
@@ -45,6 +46,11 @@ class ScaError(RuntimeError):
     def __init__(self, code: int, message: str):
         super().__init__(f"libsca error {code}: {message}")
         self.code = code
+
+
+class sca_mask_options(ctypes.Structure):
+    _fields_ = [("textq_policy", ctypes.c_int32), ("history_segments", ctypes.c_int32),
+                ("keep_blocks", ctypes.c_void_p), ("keep_blocks_len", ctypes.c_int64)]
 
 
 class sca_segment(ctypes.Structure):
@@ -62,6 +68,9 @@ _SIGS = {
     "sca_metadata_create": [ctypes.POINTER(_P)],
     "sca_build_segment_mask_metadata": [_P, ctypes.POINTER(sca_segment), _i32,
                                         ctypes.POINTER(sca_segment), _i32, _i32],
+    "sca_build_segment_mask_metadata_ex": [_P, ctypes.POINTER(sca_segment), _i32,
+                                           ctypes.POINTER(sca_segment), _i32,
+                                           ctypes.POINTER(sca_mask_options)],
     "sca_metadata_get_counts": [_P, _pi64, _pi64, _pi64, _pi32, _pi32, _pi64, _pi64, _pi64],
     "sca_metadata_get_schedule": [_P, ctypes.POINTER(_pi32), ctypes.POINTER(_pi32),
                                   ctypes.POINTER(ctypes.POINTER(ctypes.c_uint8))],
@@ -156,10 +165,24 @@ class Metadata:
             _lib.sca_metadata_destroy(self.handle)
             self.handle = None
 
-    def build(self, cached: Sequence, current: Sequence, textq_policy: int = TEXTQ_OWN_TAIL):
+    def build(self, cached: Sequence, current: Sequence, textq_policy: int = TEXTQ_OWN_TAIL,
+              history_segments: int = -1, keep_blocks=None):
+        """``keep_blocks``: None, or a [query tiles, key tiles] array of bools
+        / 0-1 bytes (a 0 drops that video-only key tile for that query tile)."""
         c, u = _SegArray(cached), _SegArray(current)
-        _check(_lib.sca_build_segment_mask_metadata(self.handle, c.arr, c.n, u.arr, u.n,
-                                                    int(textq_policy)))
+        if history_segments == -1 and keep_blocks is None:
+            _check(_lib.sca_build_segment_mask_metadata(self.handle, c.arr, c.n, u.arr, u.n,
+                                                        int(textq_policy)))
+            return self
+        keep = None
+        if keep_blocks is not None:
+            import numpy as np
+            keep = np.ascontiguousarray(np.asarray(keep_blocks).astype(np.uint8).ravel())
+        opt = sca_mask_options(int(textq_policy), int(history_segments),
+                               keep.ctypes.data if keep is not None else None,
+                               int(keep.size) if keep is not None else 0)
+        _check(_lib.sca_build_segment_mask_metadata_ex(self.handle, c.arr, c.n, u.arr, u.n,
+                                                       ctypes.byref(opt)))
         return self
 
     def counts(self) -> dict:
@@ -203,8 +226,17 @@ class Metadata:
 
 def build_segment_mask_metadata(cached: Sequence, current: Sequence,
                                 textq_policy: int = TEXTQ_OWN_TAIL,
-                                md: Optional[Metadata] = None) -> Metadata:
-    return (md or Metadata()).build(cached, current, textq_policy)
+                                md: Optional[Metadata] = None, history_segments: int = -1,
+                                keep_blocks=None) -> Metadata:
+    return (md or Metadata()).build(cached, current, textq_policy, history_segments,
+                                    keep_blocks)
+
+
+def build_for(problem, md: Optional[Metadata] = None) -> Metadata:
+    """Metadata of a workloads.Problem (its policy, window and kept blocks)."""
+    return build_segment_mask_metadata(problem.cached, problem.current, problem.textq_policy, md,
+                                       getattr(problem, "history_segments", -1),
+                                       getattr(problem, "keep_blocks", None))
 
 
 def metadata_upload(md: Metadata, stream=None) -> Metadata:

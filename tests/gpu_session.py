@@ -36,8 +36,7 @@ class GpuSession:
         self.q = inputs["q"].to(self.dev).contiguous()
         self.k_cur = inputs["k_cur"].to(self.dev).contiguous()
         self.v_cur = inputs["v_cur"].to(self.dev).contiguous()
-        self.md = sca.build_segment_mask_metadata(problem.cached, problem.current,
-                                                  problem.textq_policy).upload()
+        self.md = sca.build_for(problem).upload()
         self.status = torch.zeros(1, dtype=torch.int32, device=self.dev)
 
     def forward(self, q=None, k_cur=None, v_cur=None, workspace=True):

@@ -22,7 +22,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _builder(p):
-    return sca.build_segment_mask_metadata(p.cached, p.current, p.textq_policy)
+    return sca.build_for(p)
 
 
 def _overlap_problem():
@@ -64,6 +64,40 @@ def test_schedule_descriptors_and_count_small(p):
     kd, qd = md.descriptors()
     assert np.array_equal(kd, ocache.key_descriptors(p.current, len(p.cached)))
     assert np.array_equal(qd, ocache.query_descriptors(lay))
+
+
+def _window_and_blocks():
+    sess = W.small_session(heads=1)
+    long_sess = W.Problem("long-small", tuple(W.small_packed(seed=5, n_segments=7).current),
+                          (W.Segment(3, 60, 9, (W.Action(4, 0, 2), W.Action(6, 1, 3))),), heads=1)
+    return [W.with_history(sess, 0), W.with_history(sess, 1), W.with_history(long_sess, 3),
+            W.with_history(W.small_packed(seed=21, n_segments=14), 2),
+            W.with_random_blocks(long_sess, 0.25, 7),
+            W.with_random_blocks(W.with_history(long_sess, 4), 0.5, 8),
+            W.with_random_blocks(W.small_packed(seed=21, n_segments=14), 0.3, 9),
+            W.with_random_blocks(W.with_history(W.session_480p_single_turn(), 2), 0.25, 10)]
+
+
+@pytest.mark.parametrize("p", _window_and_blocks(), ids=lambda p: p.name)
+def test_window_and_dropped_blocks_schedule(p):
+    """Sliding window and dropped video blocks: schedule, classes and A
+    bit-exact against the oracle's brute-force tiles."""
+    lay = orule.Layout.of(p)
+    md = _builder(p)
+    c = md.counts()
+    assert c["unmasked_pairs"] == lay.unmasked_pairs()
+    row_ptr, kv, flag = md.schedule()
+    o_row_ptr, o_kv, o_flag = osched.schedule(lay)
+    assert np.array_equal(row_ptr, o_row_ptr)
+    assert np.array_equal(kv, o_kv) and np.array_equal(flag, o_flag)
+
+
+def test_window_closed_form_and_bad_keep_blocks():
+    p = W.with_history(W.session_480p_long(), 4)
+    assert _builder(p).counts()["unmasked_pairs"] == 742_096_884
+    with pytest.raises(sca.ScaError) as e:
+        sca.build_segment_mask_metadata((), (W.Segment(2, 4, 1),), keep_blocks=np.ones((3, 3)))
+    assert e.value.code == sca.ERR_INVALID_ARG and "keep_blocks" in str(e.value)
 
 
 @pytest.mark.slow

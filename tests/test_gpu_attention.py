@@ -306,3 +306,54 @@ def test_packed_360k_sampled_rows():
     o_ref, lse_ref = oattn.attention_rows(lay, q, k, v, rows, p.softmax_scale, heads=heads)
     compare(o[rows][:, heads], lse[heads][:, rows], o_ref, lse_ref)
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+
+
+def _window_blocks_problems():
+    sess = W.small_session(heads=2)
+    long_sess = W.Problem("long-small", tuple(W.small_packed(seed=5, n_segments=7).current),
+                          (W.Segment(3, 60, 9, (W.Action(4, 0, 2), W.Action(6, 1, 3))),), heads=2)
+    return [W.with_history(sess, 0), W.with_history(sess, 1), W.with_history(long_sess, 3),
+            W.with_history(W.small_packed(seed=21, n_segments=14), 2),
+            W.with_random_blocks(long_sess, 0.25, 7),
+            W.with_random_blocks(W.with_history(long_sess, 4), 0.5, 8),
+            W.with_random_blocks(W.small_packed(seed=21, n_segments=14), 0.3, 9)]
+
+
+@pytest.mark.parametrize("p", _window_blocks_problems(), ids=lambda p: p.name)
+def test_window_and_dropped_blocks_match_oracle(p):
+    """Sliding window over earlier segments and dropped video blocks: the
+    kernel (window in its predicate, blocks removed from the schedule)
+    against the oracle's explicit mask; and the mask probe on the same
+    layouts (forbidden key classes read exactly 0)."""
+    inputs = W.make_inputs(p, 44, 2.0)
+    s = GpuSession(p, inputs)
+    o, lse = s.forward()
+    q, k, v = oracle_inputs(inputs)
+    lay = orule.Layout.of(p)
+    o_ref, lse_ref = oattn.attention(lay, q, k, v, p.softmax_scale)
+    compare(o, lse, o_ref, lse_ref)
+    # exact zeros on every key the window or a dropped block hides
+    ones = torch.ones(lay.n_keys, p.heads, 128, dtype=torch.bfloat16)
+    m = lay.mask()
+    hidden = torch.from_numpy(~m.any(axis=0))          # keys no query sees
+    probe_v = torch.zeros_like(ones)
+    probe_v[hidden] = 1.0
+    probe_v[~hidden, :, 1] = 1.0
+    nc = p.n_cache_tokens
+    s2 = GpuSession(p, dict(inputs, cache_v=probe_v[:nc].contiguous(), v_cur=probe_v[nc:].contiguous()))
+    o2, _ = s2.forward()
+    assert torch.all(o2[..., 0].float() == 0.0)
+
+
+@pytest.mark.slow
+def test_full_size_window_and_sparse_blocks():
+    p = W.with_random_blocks(W.with_history(W.session_480p_long(), 4), 0.25, 11)
+    inputs = W.make_inputs(p, 45)
+    s = GpuSession(p, inputs)
+    o, lse = s.forward()
+    rows = W.sample_rows(p.n_query_tokens, 40, seed=3)
+    heads = [1, 9]
+    q, k, v = oracle_inputs(inputs)
+    lay = orule.Layout.of(p)
+    o_ref, lse_ref = oattn.attention_rows(lay, q, k, v, rows, p.softmax_scale, heads=heads)
+    compare(o[rows][:, heads], lse[heads][:, rows], o_ref, lse_ref)
