@@ -41,9 +41,11 @@ WORKLOADS = {
     "packed-360k": W.packed_360k,
     "tiny-packed": W.tiny_packed,
     # inference options (sliding window of 4 earlier segments; a quarter of
-    # the video blocks kept, drawn at random with a fixed seed)
+    # the video blocks kept, drawn at random with a fixed seed per pair of
+    # query tiles)
     "480p-long-session-window4": lambda: W.with_history(W.session_480p_long(), 4),
-    "480p-long-session-blocks25": lambda: W.with_random_blocks(W.session_480p_long(), 0.25, 25),
+    "480p-long-session-blocks25": lambda: W.with_random_blocks(W.session_480p_long(), 0.25, 25,
+                                                               group=2),
 }
 KERNEL_SOURCES = ["segment_causal_masked_b200/csrc/sca_kernels.cu",
                   "segment_causal_masked_b200/csrc/sca_internal.h"]

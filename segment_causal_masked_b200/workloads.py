@@ -221,13 +221,18 @@ def n_key_tiles(problem: Problem) -> int:
     return (problem.n_cache_tokens + 127) // 128 + (problem.n_query_tokens + 127) // 128
 
 
-def with_random_blocks(problem: Problem, keep: float, seed: int) -> Problem:
-    """The same call keeping a seeded random fraction ``keep`` of each query
-    tile's key tiles (only video-only key tiles can be dropped; the others
-    are kept whatever the draw)."""
+def with_random_blocks(problem: Problem, keep: float, seed: int, group: int = 1) -> Problem:
+    """The same call keeping a seeded random fraction ``keep`` of the key
+    tiles, drawn once per ``group`` consecutive query tiles (neighbouring
+    query tiles sharing their kept blocks, as a score-based selection
+    tends to). Only video-only key tiles can be dropped; the others are kept
+    whatever the draw."""
     rng = np.random.default_rng(seed)
-    mask = rng.random((n_query_tiles(problem), n_key_tiles(problem))) < keep
-    return dataclasses.replace(problem, name=f"{problem.name}-blocks{int(round(100 * keep))}",
+    n_qt = n_query_tiles(problem)
+    draw = rng.random(((n_qt + group - 1) // group, n_key_tiles(problem))) < keep
+    mask = np.repeat(draw, group, axis=0)[:n_qt]
+    return dataclasses.replace(problem, name=f"{problem.name}-blocks{int(round(100 * keep))}"
+                                            + (f"g{group}" if group > 1 else ""),
                                keep_blocks=mask)
 
 
