@@ -90,3 +90,41 @@ def append(cache_k: np.ndarray, cache_v: np.ndarray, cache_desc: np.ndarray,
     cv[:, length:length + n, :] = np.transpose(v, (1, 0, 2))
     cd[length:length + n] = segment_key_descriptors(segment, segment_index)
     return ck, cv, cd, length + n
+
+
+# ---------------------------------------------------------------------------
+# INT8 cache
+# ---------------------------------------------------------------------------
+# The pages quantise the KV cache to INT8 for single-GPU inference ([picx]
+# "Inference") without giving the scheme. Reading: every 128-value row of K
+# or V (one token, one head) is quantised symmetrically with its own scale,
+#     scale = max_d |x_d| / 127        (float32)
+#     q_d   = round_half_even(x_d / scale), clamped to [-127, 127]   (int8)
+# with x the bf16 value widened to float32 and both divisions in float32
+# (a row of zeros has scale 0 and q = 0). The cached value is q * scale.
+
+def quantize_rows(x: np.ndarray):
+    """x: [..., 128] (bf16 values as float32). Returns (q int8 [..., 128],
+    scale float32 [...])."""
+    x = np.asarray(x, dtype=np.float32)
+    amax = np.abs(x).max(axis=-1)
+    scale = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    q = np.rint((x / safe[..., None]).astype(np.float32))
+    q = np.clip(q, -127, 127).astype(np.int8)
+    q[scale == 0] = 0
+    return q, scale
+
+
+def dequantize_rows(q: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    return q.astype(np.float64) * scale.astype(np.float64)[..., None]
+
+
+def append_int8(cache_q: np.ndarray, cache_scale: np.ndarray, length: int, k: np.ndarray):
+    """Quantise token-major [n, H, 128] rows into the head-major int8 cache
+    [H, capacity, 128] and its scales [H, capacity] at rows [length, length+n)."""
+    q, s = quantize_rows(np.transpose(k, (1, 0, 2)))
+    cq, cs = cache_q.copy(), cache_scale.copy()
+    cq[:, length:length + k.shape[0], :] = q
+    cs[:, length:length + k.shape[0]] = s
+    return cq, cs
