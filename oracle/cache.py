@@ -101,7 +101,9 @@ def append(cache_k: np.ndarray, cache_v: np.ndarray, cache_desc: np.ndarray,
 #     scale = max_d |x_d| / 127        (float32)
 #     q_d   = round_half_even(x_d / scale), clamped to [-127, 127]   (int8)
 # with x the bf16 value widened to float32 and both divisions in float32
-# (a row of zeros has scale 0 and q = 0). The cached value is q * scale.
+# (a row of zeros has scale 0 and q = 0). The cached value is q * scale,
+# formed in float32 and rounded to bf16: dequantisation gives back a tensor
+# of the dtype the cache held before quantisation.
 
 def quantize_rows(x: np.ndarray):
     """x: [..., 128] (bf16 values as float32). Returns (q int8 [..., 128],
@@ -116,8 +118,19 @@ def quantize_rows(x: np.ndarray):
     return q, scale
 
 
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """float32 -> nearest bf16 (ties to even), returned as float32. bf16 keeps
+    the top 16 bits of a float32; rounding adds half of the dropped range,
+    minus one when the kept part is even, before truncating (finite x)."""
+    b = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    b = (b + 0x7FFF + ((b >> 16) & 1)) & 0xFFFF0000
+    return b.astype(np.uint32).view(np.float32)
+
+
 def dequantize_rows(q: np.ndarray, scale: np.ndarray) -> np.ndarray:
-    return q.astype(np.float64) * scale.astype(np.float64)[..., None]
+    """bf16(float32(q * scale)), as float64."""
+    v = q.astype(np.float32) * scale.astype(np.float32)[..., None]
+    return round_bf16(v).astype(np.float64)
 
 
 def append_int8(cache_q: np.ndarray, cache_scale: np.ndarray, length: int, k: np.ndarray):
