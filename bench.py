@@ -19,6 +19,7 @@ the slowest rank's device time.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -46,7 +47,11 @@ WORKLOADS = {
     "480p-long-session-window4": lambda: W.with_history(W.session_480p_long(), 4),
     "480p-long-session-blocks25": lambda: W.with_random_blocks(W.session_480p_long(), 0.25, 25,
                                                                group=2),
+    # INT8 KV cache (codes + per-row scales, quantised by the append kernel)
+    "480p-long-session-int8": lambda: dataclasses.replace(W.session_480p_long(),
+                                                          name="480p-long-session-int8"),
 }
+INT8_WORKLOADS = {"480p-long-session-int8"}
 KERNEL_SOURCES = ["segment_causal_masked_b200/csrc/sca_kernels.cu",
                   "segment_causal_masked_b200/csrc/sca_internal.h"]
 
@@ -150,10 +155,11 @@ class OracleSample:
     """The oracle on `rows` query rows (spread evenly over the query tiles) and
     `heads` head(s) of the workload, inputs drawn once."""
 
-    def __init__(self, problem, rows: int, heads: int = 1, seed: int = 7):
+    def __init__(self, problem, rows: int, heads: int = 1, seed: int = 7, int8: bool = False):
         import numpy as np
         import torch
 
+        from oracle import cache as ocache
         from oracle import rule as orule
 
         torch.set_num_threads(os.cpu_count() or 1)
@@ -164,6 +170,10 @@ class OracleSample:
         self.q = W.randn_bf16((nq, heads, W.HEAD_DIM), 1000 * seed).float().numpy()
         self.k = W.randn_bf16((nk, heads, W.HEAD_DIM), 1000 * seed + 1).float().numpy()
         self.v = W.randn_bf16((nk, heads, W.HEAD_DIM), 1000 * seed + 2).float().numpy()
+        if int8:   # the cached rows as the INT8 cache holds them (quantised before timing)
+            nc = problem.n_cache_tokens
+            self.k[:nc] = ocache.dequantize_rows(*ocache.quantize_rows(self.k[:nc]))
+            self.v[:nc] = ocache.dequantize_rows(*ocache.quantize_rows(self.v[:nc]))
         self.pairs = sum(sum(b - a for a, b in self.lay.ranges(int(r))) for r in self.rows)
         self.flops = 4.0 * W.HEAD_DIM * heads * self.pairs
         self.desc = (f"oracle (float64 NumPy) on {rows} query rows x {heads} head(s) of "
@@ -194,7 +204,7 @@ def run_reference(args, problem):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    sample = OracleSample(problem, args.oracle_rows)
+    sample = OracleSample(problem, args.oracle_rows, int8=args.workload in INT8_WORKLOADS)
     for _ in range(args.warmup):
         sample.run()
     secs = [sample.run() for _ in range(args.steps)]
@@ -243,7 +253,7 @@ class Session:
     """One replica of the workload on the current device: a cache holding the
     prior segments, the current segment's Q/K/V, outputs and metadata."""
 
-    def __init__(self, problem, seed: int):
+    def __init__(self, problem, seed: int, int8: bool = False):
         import torch
 
         from segment_causal_masked_b200 import sca
@@ -252,14 +262,23 @@ class Session:
         self.p = problem
         dev = torch.device("cuda", torch.cuda.current_device())
         h, nc, nq = problem.heads, problem.n_cache_tokens, problem.n_query_tokens
-        self.capacity = nc + nq
+        self.capacity = (nc + nq + 3) // 4 * 4
         g = torch.Generator(device=dev)
         g.manual_seed(seed)
         bf = torch.bfloat16
-        self.k_buf = torch.empty(h, self.capacity, 128, dtype=bf, device=dev)
-        self.v_buf = torch.empty_like(self.k_buf)
         self.desc = torch.zeros((self.capacity + 127) // 128 * 128, dtype=torch.int32, device=dev)
-        self.cache = sca.KVCache(h, self.capacity, self.k_buf, self.v_buf, self.desc)
+        if int8:
+            self.k_buf = torch.empty(h, self.capacity, 128, dtype=torch.int8, device=dev)
+            self.v_buf = torch.empty_like(self.k_buf)
+            self.k_scale = torch.empty(h, self.capacity, dtype=torch.float32, device=dev)
+            self.v_scale = torch.empty_like(self.k_scale)
+            self.cache = sca.KVCache(h, self.capacity, self.k_buf, self.v_buf, self.desc,
+                                     self.k_scale, self.v_scale)
+        else:
+            self.k_buf = torch.empty(h, self.capacity, 128, dtype=bf, device=dev)
+            self.v_buf = torch.empty_like(self.k_buf)
+            self.cache = sca.KVCache(h, self.capacity, self.k_buf, self.v_buf, self.desc)
+        self.int8 = int8
         for seg in problem.cached:
             k = torch.randn(seg.n_tokens, h, 128, generator=g, device=dev).to(bf)
             v = torch.randn(seg.n_tokens, h, 128, generator=g, device=dev).to(bf)
@@ -326,7 +345,8 @@ def run_native(args, problem):
     def max_over_ranks(x: float) -> float:
         return reduce_max(x, world, "cuda")
 
-    sess = Session(problem, seed=1000 * 2 + rank)
+    int8 = args.workload in INT8_WORKLOADS
+    sess = Session(problem, seed=1000 * 2 + rank, int8=int8)
     from segment_causal_masked_b200 import sca
     sca_md = sca.build_for(problem)
     counts = sca_md.counts()
@@ -407,8 +427,9 @@ def run_native(args, problem):
                        "effective_flop_per_step": flops,
                        "step": ("metadata build+upload, attention forward, kv_cache_append"
                                 if sess.appends else "metadata build+upload, attention forward"),
+                       "kv_cache": "int8 codes + fp32 row scales" if int8 else "bf16",
                        "l2": "inputs larger than L2 (cached K/V %.2f GB per tensor)"
-                             % (problem.n_cache_tokens * h * 256 / 1e9),
+                             % (problem.n_cache_tokens * h * (132 if int8 else 256) / 1e9),
                        "parallelism": f"replicas x{world}",
                        "split_plan": sess.plan},
             "pct_of_peak": 100.0 * value / world / peak,
@@ -422,7 +443,7 @@ def run_native(args, problem):
             "clocks": clock_info,
         }
         if not args.no_cpu_baseline:
-            sample = OracleSample(problem, args.baseline_rows)
+            sample = OracleSample(problem, args.baseline_rows, int8=int8)
             dt = sample.run()
             line["cpu_baseline"] = {"value": sample.flops / dt / 1e12, "unit": "TFLOP/s",
                                     "cores": cpu_threads(), "kind": "oracle",

@@ -203,6 +203,27 @@ SCA_API void sca_metadata_destroy(sca_metadata* md);
 SCA_API int sca_kv_cache_create(sca_kv_cache** out, int32_t heads, int32_t head_dim,
                         int64_t capacity, void* k_buf, void* v_buf, void* desc_buf);
 
+/* INT8 KV cache (Hy-Nomas summary on picx.dev, "Inference": the cache may be
+ * quantised to INT8 for single-GPU inference; the pages give no scheme).
+ * Each 128-value row of K or V (one token, one head) is stored as int8 codes
+ * with one fp32 scale:
+ *     scale = max_d |x_d| / 127,   code_d = round_half_even(x_d / scale)
+ * in fp32 from the bf16 values (a zero row: scale 0, codes 0), clamped to
+ * [-127, 127]; the cached value is code * scale. Caller-owned buffers:
+ *   k_codes, v_codes: int8 (two's complement) [heads][capacity][128];
+ *   k_scale, v_scale: fp32 [heads][capacity];
+ *   desc_buf:         uint32 [round_up(capacity, 128)] as above.
+ * capacity must be a multiple of 4 (the scale rows are read with 16-byte
+ * aligned tensor copies): SCA_ERR_INVALID_ARG otherwise. The buffers must be
+ * 16-byte aligned (SCA_ERR_MISALIGNED). sca_kv_cache_append quantises while
+ * it copies (bit for bit the rule above); attention reads the codes and
+ * scales and dequantises tile by tile in shared memory, with the scaled
+ * value rounded to bf16 before the products. Appending and truncating work
+ * as for a bf16 cache. */
+SCA_API int sca_kv_cache_create_int8(sca_kv_cache** out, int32_t heads, int32_t head_dim,
+                                     int64_t capacity, void* k_codes, void* v_codes,
+                                     float* k_scale, float* v_scale, void* desc_buf);
+
 /* Append one segment: copy its keys and values k, v (bf16 token-major
  * [n][heads][128], n = the segment's token count) into cache rows
  * [length, length + n) of every head with 16-byte coalesced stores, write its

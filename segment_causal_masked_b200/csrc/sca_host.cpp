@@ -541,6 +541,36 @@ int sca_kv_cache_create(sca_kv_cache** out, int32_t heads, int32_t head_dim, int
   return SCA_OK;
 }
 
+int sca_kv_cache_create_int8(sca_kv_cache** out, int32_t heads, int32_t head_dim,
+                             int64_t capacity, void* k_codes, void* v_codes, float* k_scale,
+                             float* v_scale, void* desc_buf) {
+  if (!out) return fail(SCA_ERR_INVALID_ARG, "null output pointer");
+  *out = nullptr;
+  if (head_dim != SCA_HEAD_DIM) return fail(SCA_ERR_UNSUPPORTED, "head_dim must be 128");
+  if (heads < 1 || capacity < 1 || capacity > (int64_t(1) << 31) - 1)
+    return fail(SCA_ERR_INVALID_ARG, "need heads >= 1 and 1 <= capacity < 2^31");
+  if (capacity % 4)
+    return fail(SCA_ERR_INVALID_ARG, "an INT8 cache needs a capacity that is a multiple of 4 (got %lld)",
+                (long long)capacity);
+  if (!k_codes || !v_codes || !k_scale || !v_scale || !desc_buf)
+    return fail(SCA_ERR_INVALID_ARG, "null cache buffer");
+  if (!aligned16(k_codes) || !aligned16(v_codes) || !aligned16(k_scale) || !aligned16(v_scale) ||
+      !aligned16(desc_buf))
+    return fail(SCA_ERR_MISALIGNED, "cache buffers must be 16-byte aligned");
+  sca_kv_cache* c = new (std::nothrow) sca_kv_cache();
+  if (!c) return fail(SCA_ERR_INVALID_ARG, "out of host memory");
+  c->heads = heads;
+  c->capacity = capacity;
+  c->int8 = true;
+  c->k = k_codes;
+  c->v = v_codes;
+  c->k_scale = k_scale;
+  c->v_scale = v_scale;
+  c->desc = static_cast<uint32_t*>(desc_buf);
+  *out = c;
+  return SCA_OK;
+}
+
 void sca_kv_cache_destroy(sca_kv_cache* c) { delete c; }
 
 int sca_kv_cache_get(const sca_kv_cache* c, int64_t* length, int32_t* n_segments) {
@@ -579,6 +609,9 @@ int sca_kv_cache_append(sca_kv_cache* c, const sca_segment* segment, const void*
   a.v = v;
   a.k_cache = c->k;
   a.v_cache = c->v;
+  a.k_scale = c->k_scale;
+  a.v_scale = c->v_scale;
+  a.int8 = c->int8 ? 1 : 0;
   a.desc = c->desc;
   a.length = c->length;
   a.capacity = c->capacity;
@@ -636,6 +669,40 @@ static int make_map(CUtensorMap* m, const void* base, uint64_t dim1, uint64_t di
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SCA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return SCA_OK;
+}
+
+// INT8 cache codes [heads][capacity][128] viewed as 3-D (128 bytes, rows,
+// heads); box (128, 128, 1), 128-byte swizzle (one box row is one swizzle
+// span). Rows at and past `rows` read as zeros.
+static int make_code_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t heads,
+                         uint64_t capacity) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(SCA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {SCA_HEAD_DIM, rows, heads};
+  cuuint64_t strides[2] = {SCA_HEAD_DIM, capacity * SCA_HEAD_DIM};
+  cuuint32_t box[3] = {SCA_HEAD_DIM, SCA_TILE, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SCA_ERR_CUDA, "cuTensorMapEncodeTiled (codes) failed (%d)", int(r));
+  return SCA_OK;
+}
+
+// INT8 cache scales [heads][capacity] fp32 as 2-D (rows, heads); box (128, 1).
+static int make_scale_map(CUtensorMap* m, const float* base, uint64_t rows, uint64_t heads,
+                          uint64_t capacity) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(SCA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {rows, heads};
+  cuuint64_t strides[1] = {capacity * 4};
+  cuuint32_t box[2] = {SCA_TILE, 1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SCA_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", int(r));
   return SCA_OK;
 }
 
@@ -798,7 +865,14 @@ int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md
   int rc = make_map(&maps.q, q, uint64_t(heads), uint64_t(md->n_q), SCA_HEAD_DIM * 2, row, 1, SCA_TILE);
   if (!rc) rc = make_map(&maps.k_cur, k_cur, uint64_t(heads), uint64_t(md->n_q), SCA_HEAD_DIM * 2, row, 1, SCA_TILE);
   if (!rc) rc = make_map(&maps.v_cur, v_cur, uint64_t(heads), uint64_t(md->n_q), SCA_HEAD_DIM * 2, row, 1, SCA_TILE);
-  if (!rc && md->n_cache > 0) {
+  const bool int8_cache = md->n_cache > 0 && cache->int8;
+  if (!rc && int8_cache) {
+    const uint64_t n = uint64_t(md->n_cache), cap = uint64_t(cache->capacity);
+    rc = make_code_map(&maps.k_cache, cache->k, n, uint64_t(heads), cap);
+    if (!rc) rc = make_code_map(&maps.v_cache, cache->v, n, uint64_t(heads), cap);
+    if (!rc) rc = make_scale_map(&maps.k_scale, cache->k_scale, n, uint64_t(heads), cap);
+    if (!rc) rc = make_scale_map(&maps.v_scale, cache->v_scale, n, uint64_t(heads), cap);
+  } else if (!rc && md->n_cache > 0) {
     const uint64_t hstride = uint64_t(cache->capacity) * SCA_HEAD_DIM * 2;
     rc = make_map(&maps.k_cache, cache->k, uint64_t(md->n_cache), uint64_t(heads), SCA_HEAD_DIM * 2,
                   hstride, SCA_TILE, 1);
@@ -836,7 +910,7 @@ int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md
     a.part_o = static_cast<float*>(workspace);
     a.part_ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + slots * 256 * 128 * 4);
   }
-  if (int rc2 = check_cuda(launch_attention(maps, a, static_cast<cudaStream_t>(stream)),
+  if (int rc2 = check_cuda(launch_attention(maps, a, int8_cache, static_cast<cudaStream_t>(stream)),
                            "attention launch"))
     return rc2;
   if (split)

@@ -86,11 +86,14 @@ struct AttnArgs {
   unsigned long long timeout_ns;
 };
 
+// For an INT8 cache, k_cache / v_cache cover the int8 codes (rows of 128
+// bytes) and k_scale / v_scale the per-row fp32 scales.
 struct AttnMaps {
-  CUtensorMap q, k_cur, v_cur, k_cache, v_cache;
+  CUtensorMap q, k_cur, v_cur, k_cache, v_cache, k_scale, v_scale;
 };
 
-cudaError_t launch_attention(const AttnMaps& maps, const AttnArgs& args, cudaStream_t stream);
+cudaError_t launch_attention(const AttnMaps& maps, const AttnArgs& args, bool int8_cache,
+                             cudaStream_t stream);
 cudaError_t launch_merge(const AttnArgs& args, cudaStream_t stream);
 
 // bytes of one partial slot: O [256][128] fp32 + (m, l) [256]
@@ -101,6 +104,9 @@ struct AppendArgs {
   const void* v;
   void* k_cache;
   void* v_cache;
+  float* k_scale;       // INT8 cache: per-row scales (k_cache / v_cache hold codes)
+  float* v_scale;
+  int32_t int8;         // 0: bf16 cache, 1: INT8 cache
   uint32_t* desc;
   int64_t length;       // first row written
   int64_t capacity;
@@ -119,7 +125,7 @@ cudaError_t launch_bounded_wait(int32_t* status, unsigned long long timeout_ns,
 cudaError_t launch_exp2_eval(const float* x, float* y_poly, float* y_mufu, int64_t n,
                              cudaStream_t stream);
 
-size_t attention_smem_bytes();
+size_t attention_smem_bytes(bool int8_cache);
 
 }  // namespace sca
 
@@ -169,8 +175,11 @@ struct sca_metadata {
 struct sca_kv_cache {
   int32_t heads = 0;
   int64_t capacity = 0;
-  void* k = nullptr;
+  bool int8 = false;          // codes + scales instead of bf16 rows
+  void* k = nullptr;          // bf16 rows, or int8 codes
   void* v = nullptr;
+  float* k_scale = nullptr;   // INT8 only
+  float* v_scale = nullptr;
   uint32_t* desc = nullptr;
   int64_t length = 0;
   std::vector<sca::SegLayout> segs;

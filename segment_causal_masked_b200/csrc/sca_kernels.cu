@@ -37,6 +37,25 @@ namespace sca {
 // kv_cache_append
 // ---------------------------------------------------------------------------
 
+// Descriptor word of every appended token (tails marked dead).
+__device__ __forceinline__ void append_descriptors(const AppendArgs& a) {
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; t < a.n; t += stride) {
+    uint32_t d;
+    if (t < a.n_video) {
+      d = a.seg_index | SCA_DESC_ALIVE;
+    } else if (t < int64_t(a.n_video) + a.head_len) {
+      d = a.seg_index | SCA_DESC_ALIVE | SCA_DESC_HEAD;
+    } else {
+      const int32_t r = int32_t(t - a.n_video - a.head_len);
+      int act = 0;
+      while (act + 1 < a.n_act && r >= a.tail_start[act + 1]) ++act;
+      d = a.seg_index | SCA_DESC_TAIL | (uint32_t(act) << SCA_DESC_ACTION_SHIFT);  // dead later
+    }
+    a.desc[a.length + t] = d;
+  }
+}
+
 __global__ void __launch_bounds__(256) kv_append_kernel(const AppendArgs a) {
   const uint4* __restrict__ k = static_cast<const uint4*>(a.k);
   const uint4* __restrict__ v = static_cast<const uint4*>(a.v);
@@ -55,20 +74,61 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendArgs a) {
     kc[dst] = kk;
     vc[dst] = vv;
   }
-  for (int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; t < a.n; t += stride) {
-    uint32_t d;
-    if (t < a.n_video) {
-      d = a.seg_index | SCA_DESC_ALIVE;
-    } else if (t < int64_t(a.n_video) + a.head_len) {
-      d = a.seg_index | SCA_DESC_ALIVE | SCA_DESC_HEAD;
-    } else {
-      const int32_t r = int32_t(t - a.n_video - a.head_len);
-      int act = 0;
-      while (act + 1 < a.n_act && r >= a.tail_start[act + 1]) ++act;
-      d = a.seg_index | SCA_DESC_TAIL | (uint32_t(act) << SCA_DESC_ACTION_SHIFT);  // dead later
+  append_descriptors(a);
+}
+
+// Quantise one 128-value row spread over a warp (4 values per lane, given as
+// two bf16 pairs): scale = max|x| / 127 and code = rint(x / scale) in fp32,
+// both divisions correctly rounded and the rounding to nearest even, codes
+// clamped to [-127, 127]; a zero row gets scale 0 and codes 0. Returns the
+// lane's four codes packed low byte first.
+__device__ __forceinline__ uint32_t quantize_lane(uint2 raw, float& scale) {
+  float x[4];
+  x[0] = __uint_as_float(raw.x << 16);
+  x[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+  x[2] = __uint_as_float(raw.y << 16);
+  x[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+  float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+  scale = __fdiv_rn(amax, 127.f);
+  uint32_t packed = 0;
+  if (scale > 0.f) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int qi = min(max(__float2int_rn(__fdiv_rn(x[i], scale)), -127), 127);
+      packed |= (uint32_t(qi) & 255u) << (8 * i);
     }
-    a.desc[a.length + t] = d;
   }
+  return packed;
+}
+
+// INT8 cache append: one warp per (token, head) row, K and V; 4-byte code
+// stores (a row of codes is one coalesced 128-byte line).
+__global__ void __launch_bounds__(256) kv_append_int8_kernel(const AppendArgs a) {
+  const uint2* __restrict__ k = static_cast<const uint2*>(a.k);
+  const uint2* __restrict__ v = static_cast<const uint2*>(a.v);
+  uint32_t* __restrict__ kc = static_cast<uint32_t*>(a.k_cache);
+  uint32_t* __restrict__ vc = static_cast<uint32_t*>(a.v_cache);
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = int64_t(a.n) * a.heads;
+  const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t row = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+       row += wstride) {
+    const int64_t tok = row / a.heads;
+    const int32_t h = int32_t(row - tok * a.heads);
+    const int64_t dst = int64_t(h) * a.capacity + a.length + tok;  // row of the cache
+    float sk, sv;
+    const uint32_t qk = quantize_lane(__ldg(k + row * 32 + lane), sk);
+    const uint32_t qv = quantize_lane(__ldg(v + row * 32 + lane), sv);
+    kc[dst * 32 + lane] = qk;
+    vc[dst * 32 + lane] = qv;
+    if (lane == 0) {
+      a.k_scale[dst] = sk;
+      a.v_scale[dst] = sv;
+    }
+  }
+  append_descriptors(a);
 }
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
@@ -79,7 +139,11 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
   const int64_t chunks = int64_t(a.n) * a.heads * 16;
   int64_t blocks = (chunks + 255) / 256;
   blocks = blocks < int64_t(sms) * 8 ? blocks : int64_t(sms) * 8;
-  kv_append_kernel<<<unsigned(blocks), 256, 0, stream>>>(a);
+  if (a.int8) {
+    kv_append_int8_kernel<<<unsigned(blocks), 256, 0, stream>>>(a);
+  } else {
+    kv_append_kernel<<<unsigned(blocks), 256, 0, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 
@@ -165,6 +229,25 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int32_t c0, int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// `count` arrivals at once.
+__device__ __forceinline__ void mbar_arrive_n(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+// Make this thread's shared-memory stores visible to the tensor cores.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -399,6 +482,45 @@ __device__ __forceinline__ void exp_pack_store(const float (&x)[128], uint64_t s
   }
 }
 
+// INT8 cache: dequantise row r of a staged code tile (128 rows of 128 int8
+// codes, 128-byte swizzle, as the tensor copy lays it out) into row r of a
+// bf16 operand tile in the layout the tensor copy of a bf16 tile gives (two
+// 64-column halves 16 KB apart, 128-byte swizzle). A code c becomes the exact
+// float c through the bit pattern 2^23 + (c + 128), then c * scale is rounded
+// once to fp32 and once to bf16. Both tiles start on 1024-byte boundaries,
+// so the swizzle of row r XORs the 16-byte chunk index with r & 7.
+__device__ __forceinline__ void dequant_row(const uint8_t* codes, float scale, uint8_t* tile, int r) {
+  const uint32_t sw = uint32_t(r & 7);
+  const uint64_t s2 = f2(scale, scale);
+  const uint64_t off2 = f2(-8388736.f, -8388736.f);  // -(2^23 + 128)
+  const uint64_t zero2 = f2(0.f, 0.f);
+  uint4 w[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    w[c] = *reinterpret_cast<const uint4*>(codes + r * 128 + ((uint32_t(c) ^ sw) << 4));
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {  // codes of columns 16c .. 16c + 15
+    const uint32_t words[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+    uint32_t out[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t u = words[k] ^ 0x80808080u;  // c + 128 in every byte
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const float f0 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u + 2u * b));
+        const float f1 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7541u + 2u * b));
+        float v0, v1;
+        unf2(fma2(add2(f2(f0, f1), off2), s2, zero2), v0, v1);
+        out[2 * k + b] = pack_bf16(v0, v1);
+      }
+    }
+    uint8_t* row = tile + (c >> 2) * (128 * 128) + r * 128;  // half c / 4
+    const uint32_t ch = uint32_t(2 * (c & 3));
+    *reinterpret_cast<uint4*>(row + ((ch ^ sw) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+    *reinterpret_cast<uint4*>(row + (((ch + 1u) ^ sw) << 4)) = make_uint4(out[4], out[5], out[6], out[7]);
+  }
+}
+
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -439,22 +561,40 @@ constexpr int kPolyEvery = 0;             // every n-th exponential pair of FULL
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr uint32_t kOffQ = 0;                            // Q0, Q1
 constexpr uint32_t kOffKV = 2 * kTile;                   // ring of K/V tiles
-constexpr uint32_t kOffBar = kOffKV + kStages * kTile;
+// INT8 cache only: two staged code tiles (slot 0 takes the K tiles, slot 1
+// the V tiles) and their 128 row scales
+constexpr uint32_t kCodeTile = 128 * 128;                // 16 KB
+constexpr uint32_t kOffCodes = kOffKV + kStages * kTile;
+constexpr uint32_t kOffScales = kOffCodes + 2 * kCodeTile;
+constexpr uint32_t kScaleBytes = 128 * 4;
+__host__ __device__ constexpr uint32_t off_bar(bool int8) { return int8 ? kOffScales + 2 * kScaleBytes : kOffCodes; }
 constexpr uint32_t kBarQ = 0, kBarFull = 1, kBarEmpty = kBarFull + kStages,
                    kBarS = kBarEmpty + kStages, kBarP = kBarS + 2, kBarO = kBarP + 2,
-                   kBarDrain = kBarO + 2, kNumBars = kBarDrain + 1;
-constexpr uint32_t kOffCtl = kOffBar + kNumBars * 8;
-constexpr uint32_t kOffTmemSlot = kOffCtl + 16;
-constexpr uint32_t kSmemBytes = kOffTmemSlot + 16 + 1024;  // + alignment slack
+                   kBarDrain = kBarO + 2, kBarCodeFull = kBarDrain + 1,
+                   kBarCodeEmpty = kBarCodeFull + 2, kNumBars = kBarCodeEmpty + 2;
+__host__ __device__ constexpr uint32_t smem_bytes(bool int8) {
+  return off_bar(int8) + kNumBars * 8 + 16 + 16 + 1024;  // bars, control, TMEM slot, alignment slack
+}
+static_assert(smem_bytes(true) <= 232448, "the INT8 layout must fit the 227 KB a CTA may use");
 
-size_t attention_smem_bytes() { return kSmemBytes; }
+size_t attention_smem_bytes(bool int8_cache) { return smem_bytes(int8_cache); }
 
+// kInt8: the cache holds int8 codes with per-row scales (tm_kcache and
+// tm_vcache cover the codes, tm_kscale and tm_vscale the scales); the softmax
+// warpgroups dequantise the cache tiles into the operand ring one step ahead
+// of the MMAs. Otherwise the cache is bf16 and the scale maps are unused.
+template <bool kInt8>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_kcur,
                     const __grid_constant__ CUtensorMap tm_vcur,
                     const __grid_constant__ CUtensorMap tm_kcache,
-                    const __grid_constant__ CUtensorMap tm_vcache, const AttnArgs p) {
+                    const __grid_constant__ CUtensorMap tm_vcache,
+                    const __grid_constant__ CUtensorMap tm_kscale,
+                    const __grid_constant__ CUtensorMap tm_vscale, const AttnArgs p) {
+  constexpr uint32_t kOffBar = off_bar(kInt8);
+  constexpr uint32_t kOffCtl = kOffBar + kNumBars * 8;
+  constexpr uint32_t kOffTmemSlot = kOffCtl + 16;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -488,8 +628,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     ctl->abort = 0;
     mbar_init(bar(kBarQ), 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(kBarFull + s), 1);
+      // INT8: a dequantised tile is complete after its warpgroup's 128 arrivals
+      mbar_init(bar(kBarFull + s), kInt8 ? 128 : 1);
       mbar_init(bar(kBarEmpty + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBarCodeFull + s), 1);
+      mbar_init(bar(kBarCodeEmpty + s), 128);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(kBarS + t), 1);
@@ -526,9 +671,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(sQ + kTile + kHalf, &tm_q, bar(kBarQ), 64, head, q_row0 + 128);
       int it = 0;
       bool ok = true;
+      // INT8: the cache tiles (a prefix of the ascending list) go to the code
+      // slots, where a softmax warpgroup dequantises them into the ring
+      auto staged = [&](int i) { return kInt8 && int(list[i >> 1] & kPairTileMask) < p.n_cache_tiles; };
       for (int j = 0; j < n_iter && ok; ++j) {
         const int tile = int(list[j] & kPairTileMask);
         for (int kv = 0; kv < 2; ++kv, ++it) {
+          if (staged(it)) {
+            const uint32_t cb = bar(kBarCodeFull + kv);
+            if (!wait_bar(bar(kBarCodeEmpty + kv), (uint32_t(it >> 1) & 1u) ^ 1u, ctl, p.status,
+                          p.timeout_ns)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(cb, kCodeTile + kScaleBytes);
+            tma_load_3d(sbase + kOffCodes + uint32_t(kv) * kCodeTile, kv ? &tm_vcache : &tm_kcache,
+                        cb, 0, tile * 128, head);
+            tma_load_2d(sbase + kOffScales + uint32_t(kv) * kScaleBytes,
+                        kv ? &tm_vscale : &tm_kscale, cb, tile * 128, head);
+            continue;
+          }
           const int s = it % kStages;
           const uint32_t ph = uint32_t(it / kStages) & 1u;
           if (!wait_bar(bar(kBarEmpty + s), ph ^ 1u, ctl, p.status, p.timeout_ns)) {
@@ -537,7 +699,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t dst = sbase + kOffKV + uint32_t(s) * kTile;
           mbar_expect_tx(bar(kBarFull + s), kTile);
-          if (tile < p.n_cache_tiles) {
+          if (kInt8) mbar_arrive_n(bar(kBarFull + s), 127);
+          if (!kInt8 && tile < p.n_cache_tiles) {
             const CUtensorMap* m = kv ? &tm_vcache : &tm_kcache;
             tma_load_3d(dst, m, bar(kBarFull + s), 0, tile * 128, head);
             tma_load_3d(dst + kHalf, m, bar(kBarFull + s), 64, tile * 128, head);
@@ -550,11 +713,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) {
-        // drain: let every armed load land before the CTA can exit
+        // drain: let every armed load land before the CTA can exit. A ring
+        // slot's latest load is among the last kStages issued; a code slot's
+        // is the last staged load of its parity (staged loads form a prefix).
         for (int back = 1; back <= kStages && it - back >= 0; ++back) {
           const int i2 = it - back;
-          wait_bounded(bar(kBarFull + i2 % kStages), uint32_t(i2 / kStages) & 1u, ctl, nullptr,
-                       p.timeout_ns);
+          if (!staged(i2)) {
+            wait_bounded(bar(kBarFull + i2 % kStages), uint32_t(i2 / kStages) & 1u, ctl, nullptr,
+                         p.timeout_ns);
+          } else if (i2 + 2 >= it || !staged(i2 + 2)) {
+            wait_bounded(bar(kBarCodeFull + (i2 & 1)), uint32_t(i2 >> 1) & 1u, ctl, nullptr,
+                         p.timeout_ns);
+          }
         }
         wait_bounded(bar(kBarQ), 0, ctl, nullptr, p.timeout_ns);
       }
@@ -642,8 +812,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool o_init = false;  // O_t holds a P V result (else its TMEM is undefined)
     bool ok = true;
     const uint64_t scale2 = f2(p.scale_log2, p.scale_log2);
+    // INT8 cache: warpgroup 1 dequantises the K tiles (it = 2j) and
+    // warpgroup 0 the V tiles (it = 2j + 1) of the list's cache prefix, each
+    // thread one row, so that after the P of step j the K of step j + 2 and
+    // the V of step j + 1 are ready (both a step before the MMAs need them).
+    int conv_it = 1 - t;  // next tile this warpgroup dequantises
+    auto convert_upto = [&](int last) -> bool {
+      for (; conv_it <= last && conv_it < 2 * n_iter; conv_it += 2) {
+        if (int(list[conv_it >> 1] & kPairTileMask) >= p.n_cache_tiles) {
+          conv_it = 2 * n_iter;  // past the prefix: nothing left to convert
+          break;
+        }
+        const int slot8 = conv_it & 1, s = conv_it % kStages;
+        bool ready = wait_bar(bar(kBarCodeFull + slot8), uint32_t(conv_it >> 1) & 1u, ctl, p.status,
+                              p.timeout_ns) &&
+                     wait_bar(bar(kBarEmpty + s), (uint32_t(conv_it / kStages) & 1u) ^ 1u, ctl,
+                              p.status, p.timeout_ns);
+        if (!__all_sync(0xFFFFFFFFu, ready)) return false;
+        const float sc = reinterpret_cast<const float*>(smem + kOffScales + slot8 * kScaleBytes)[r];
+        dequant_row(smem + kOffCodes + slot8 * kCodeTile, sc, smem + kOffKV + s * kTile, r);
+        fence_proxy_async_smem();
+        mbar_arrive(bar(kBarFull + s));
+        mbar_arrive(bar(kBarCodeEmpty + slot8));
+      }
+      return true;
+    };
+    if (kInt8 && !convert_upto(1 + t)) ok = false;
     uint32_t e_next = n_iter > 0 ? list[0] : 0u;
-    for (int j = 0; j < n_iter; ++j) {
+    for (int j = 0; ok && j < n_iter; ++j) {
       const uint32_t e = e_next;
       if (j + 1 < n_iter) e_next = list[j + 1];   // prefetch the next schedule entry
       const int tile = int(e & kPairTileMask);
@@ -734,6 +930,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kBarP + t));
+      if (kInt8 && !convert_upto(2 * j + 3 + t)) {
+        ok = false;
+        break;
+      }
     }
     // ---------------------------------------------------------- epilogue
     if (ok && n_iter > 0) ok = wait_bar(bar(kBarO + t), 0, ctl, p.status, p.timeout_ns);
@@ -801,21 +1001,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-cudaError_t launch_attention(const AttnMaps& maps, const AttnArgs& args, cudaStream_t stream) {
+template <bool kInt8>
+static cudaError_t launch_attention_t(const AttnMaps& maps, const AttnArgs& args,
+                                      cudaStream_t stream) {
   static int configured_mask = 0;
+  constexpr uint32_t kSmem = smem_bytes(kInt8);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 31 && !(configured_mask & (1 << dev))) {
-    e = cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(kSmemBytes));
+  if (dev >= 31 || !(configured_mask & (1 << dev))) {
+    e = cudaFuncSetAttribute(attn_fwd_kernel<kInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(kSmem));
     if (e != cudaSuccess) return e;
-    configured_mask |= 1 << dev;
+    if (dev < 31) configured_mask |= 1 << dev;
   }
   const unsigned grid = unsigned(args.n_full) + unsigned(args.n_split) * unsigned(args.chunks);
-  attn_fwd_kernel<<<grid, kThreads, kSmemBytes, stream>>>(maps.q, maps.k_cur, maps.v_cur,
-                                                          maps.k_cache, maps.v_cache, args);
+  attn_fwd_kernel<kInt8><<<grid, kThreads, kSmem, stream>>>(
+      maps.q, maps.k_cur, maps.v_cur, maps.k_cache, maps.v_cache, maps.k_scale, maps.v_scale, args);
   return cudaGetLastError();
+}
+
+cudaError_t launch_attention(const AttnMaps& maps, const AttnArgs& args, bool int8_cache,
+                             cudaStream_t stream) {
+  return int8_cache ? launch_attention_t<true>(maps, args, stream)
+                    : launch_attention_t<false>(maps, args, stream);
 }
 
 // ---------------------------------------------------------------------------

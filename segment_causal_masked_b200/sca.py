@@ -33,7 +33,8 @@ EXPORTED = (
     "sca_metadata_create", "sca_build_segment_mask_metadata",
     "sca_build_segment_mask_metadata_ex", "sca_metadata_get_counts",
     "sca_metadata_get_schedule", "sca_metadata_get_descriptors", "sca_metadata_upload",
-    "sca_metadata_destroy", "sca_kv_cache_create", "sca_kv_cache_append",
+    "sca_metadata_destroy", "sca_kv_cache_create", "sca_kv_cache_create_int8",
+    "sca_kv_cache_append",
     "sca_kv_cache_truncate", "sca_kv_cache_get", "sca_kv_cache_destroy",
     "sca_action_causal_attn_fwd", "sca_action_causal_attn_fwd_static_ws",
     "sca_attn_workspace_bytes", "sca_attn_plan",
@@ -79,6 +80,7 @@ _SIGS = {
     "sca_metadata_upload": [_P, _P],
     "sca_metadata_destroy": [_P],
     "sca_kv_cache_create": [ctypes.POINTER(_P), _i32, _i32, _i64, _P, _P, _P],
+    "sca_kv_cache_create_int8": [ctypes.POINTER(_P), _i32, _i32, _i64, _P, _P, _P, _P, _P],
     "sca_kv_cache_append": [_P, ctypes.POINTER(sca_segment), _P, _P, _P],
     "sca_kv_cache_truncate": [_P, _i32],
     "sca_kv_cache_get": [_P, _pi64, _pi32],
@@ -250,16 +252,26 @@ def metadata_upload(md: Metadata, stream=None) -> Metadata:
 class KVCache:
     """Owns one ``sca_kv_cache`` handle over caller-owned device buffers:
     k_buf, v_buf bf16 [heads, capacity, 128]; desc_buf uint32/int32
-    [round_up(capacity, 128)]. The buffers must outlive the cache."""
+    [round_up(capacity, 128)]. With ``k_scale`` and ``v_scale`` (fp32
+    [heads, capacity]) the cache is INT8: k_buf, v_buf then hold int8 codes
+    [heads, capacity, 128] (sca_kv_cache_create_int8). The buffers must
+    outlive the cache."""
 
-    def __init__(self, heads: int, capacity: int, k_buf, v_buf, desc_buf):
+    def __init__(self, heads: int, capacity: int, k_buf, v_buf, desc_buf, k_scale=None,
+                 v_scale=None):
         h = _P()
-        _check(_lib.sca_kv_cache_create(ctypes.byref(h), int(heads), HEAD_DIM, int(capacity),
-                                        _ptr(k_buf), _ptr(v_buf), _ptr(desc_buf)))
+        self.int8 = k_scale is not None or v_scale is not None
+        if self.int8:
+            _check(_lib.sca_kv_cache_create_int8(ctypes.byref(h), int(heads), HEAD_DIM,
+                                                 int(capacity), _ptr(k_buf), _ptr(v_buf),
+                                                 _ptr(k_scale), _ptr(v_scale), _ptr(desc_buf)))
+        else:
+            _check(_lib.sca_kv_cache_create(ctypes.byref(h), int(heads), HEAD_DIM, int(capacity),
+                                            _ptr(k_buf), _ptr(v_buf), _ptr(desc_buf)))
         self.handle = h
         self.heads = heads
         self.capacity = capacity
-        self._bufs = (k_buf, v_buf, desc_buf)
+        self._bufs = (k_buf, v_buf, desc_buf, k_scale, v_scale)
 
     def __del__(self):
         if getattr(self, "handle", None):
@@ -285,6 +297,10 @@ class KVCache:
 
 def kv_cache_create(heads, capacity, k_buf, v_buf, desc_buf) -> KVCache:
     return KVCache(heads, capacity, k_buf, v_buf, desc_buf)
+
+
+def kv_cache_create_int8(heads, capacity, k_codes, v_codes, k_scale, v_scale, desc_buf) -> KVCache:
+    return KVCache(heads, capacity, k_codes, v_codes, desc_buf, k_scale, v_scale)
 
 
 def kv_cache_append(cache: KVCache, segment, k, v, stream=None) -> None:

@@ -9,23 +9,37 @@ from __future__ import annotations
 import numpy as np
 import torch
 
+from oracle import cache as ocache
 from segment_causal_masked_b200 import sca
 from segment_causal_masked_b200 import workloads as W
 
 
 class GpuSession:
+    """``int8``: the cache stores int8 codes and per-row scales (the append
+    kernel quantises)."""
+
     def __init__(self, problem: W.Problem, inputs: dict, capacity: int = None,
-                 device: str = "cuda:0"):
+                 device: str = "cuda:0", int8: bool = False):
         self.p = problem
         self.dev = torch.device(device)
         h = problem.heads
         nc, nq = problem.n_cache_tokens, problem.n_query_tokens
         self.capacity = capacity or max(nc + nq, 1)
+        if int8:
+            self.capacity = (self.capacity + 3) // 4 * 4
         cap_pad = (self.capacity + 127) // 128 * 128
-        self.k_buf = torch.zeros(h, self.capacity, 128, dtype=torch.bfloat16, device=self.dev)
-        self.v_buf = torch.zeros_like(self.k_buf)
         self.desc = torch.zeros(cap_pad, dtype=torch.int32, device=self.dev)
-        self.cache = sca.KVCache(h, self.capacity, self.k_buf, self.v_buf, self.desc)
+        if int8:
+            self.k_buf = torch.zeros(h, self.capacity, 128, dtype=torch.int8, device=self.dev)
+            self.v_buf = torch.zeros_like(self.k_buf)
+            self.k_scale = torch.zeros(h, self.capacity, dtype=torch.float32, device=self.dev)
+            self.v_scale = torch.zeros_like(self.k_scale)
+            self.cache = sca.KVCache(h, self.capacity, self.k_buf, self.v_buf, self.desc,
+                                     self.k_scale, self.v_scale)
+        else:
+            self.k_buf = torch.zeros(h, self.capacity, 128, dtype=torch.bfloat16, device=self.dev)
+            self.v_buf = torch.zeros_like(self.k_buf)
+            self.cache = sca.KVCache(h, self.capacity, self.k_buf, self.v_buf, self.desc)
         ck = inputs["cache_k"].to(self.dev)
         cv = inputs["cache_v"].to(self.dev)
         pos = 0
@@ -59,11 +73,17 @@ class GpuSession:
         return o, lse
 
 
-def oracle_inputs(inputs: dict):
-    """float32 numpy views (exact copies of the bf16 values) for the oracle."""
+def oracle_inputs(inputs: dict, int8: bool = False):
+    """float32 numpy views (exact copies of the bf16 values) for the oracle;
+    with ``int8`` the cached keys and values are the oracle's INT8 round trip
+    (codes times scales, float64)."""
     q = inputs["q"].float().numpy()
-    k = torch.cat([inputs["cache_k"], inputs["k_cur"]]).float().numpy()
-    v = torch.cat([inputs["cache_v"], inputs["v_cur"]]).float().numpy()
+    ck, cv = inputs["cache_k"].float().numpy(), inputs["cache_v"].float().numpy()
+    if int8:
+        ck = ocache.dequantize_rows(*ocache.quantize_rows(ck))
+        cv = ocache.dequantize_rows(*ocache.quantize_rows(cv))
+    k = np.concatenate([ck, inputs["k_cur"].float().numpy()])
+    v = np.concatenate([cv, inputs["v_cur"].float().numpy()])
     return q, k, v
 
 

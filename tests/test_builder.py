@@ -183,3 +183,17 @@ def test_rebuild_replaces_contents():
     assert md.counts()["n_queries"] == 1
     md.build(W.small_session().cached, W.small_session().current)
     assert md.counts()["n_queries"] == W.small_session().n_query_tokens
+
+
+def test_int8_cache_handle_checks():
+    """The INT8 cache records caller buffers (no GPU work): capacity must be
+    a multiple of 4, buffers 16-byte aligned."""
+    base = 1 << 20   # fake, aligned device addresses: the handle never dereferences them
+    with pytest.raises(sca.ScaError) as e:
+        sca.kv_cache_create_int8(2, 6, base, base, base, base, base)
+    assert e.value.code == sca.ERR_INVALID_ARG and "multiple of 4" in str(e.value)
+    with pytest.raises(sca.ScaError) as e:
+        sca.kv_cache_create_int8(2, 8, base, base, base + 4, base, base)
+    assert e.value.code == sca.ERR_MISALIGNED
+    c = sca.kv_cache_create_int8(2, 8, base, base, base, base, base)
+    assert c.int8 and c.get() == (0, 0)
