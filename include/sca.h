@@ -262,7 +262,10 @@ SCA_API void sca_kv_cache_destroy(sca_kv_cache* cache);
  *            wave; with NULL or too little, nothing is split. The result is
  *            the same up to fp32 summation order;
  *   dev_status : device int32 (or NULL); left unchanged on success, set to
- *            SCA_ERR_DEVICE_TIMEOUT if a bounded wait in the kernel ran out;
+ *            SCA_ERR_DEVICE_TIMEOUT if a bounded wait in the kernel ran out,
+ *            or SCA_ERR_MISALIGNED if the kernel's shared-memory window did
+ *            not start close enough to a 1024-byte boundary (the INT8 cache
+ *            kernel has under 1 KB to spare; the result is then not written);
  *   stream : the caller's stream.
  * The call allocates nothing. A query that sees no key gets o = 0 and
  * lse = -inf. Calls sharing a workspace must be ordered (same stream). */

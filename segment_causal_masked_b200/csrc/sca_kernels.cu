@@ -494,13 +494,10 @@ __device__ __forceinline__ void dequant_row(const uint8_t* codes, float scale, u
   const uint64_t s2 = f2(scale, scale);
   const uint64_t off2 = f2(-8388736.f, -8388736.f);  // -(2^23 + 128)
   const uint64_t zero2 = f2(0.f, 0.f);
-  uint4 w[8];
-#pragma unroll
-  for (int c = 0; c < 8; ++c)
-    w[c] = *reinterpret_cast<const uint4*>(codes + r * 128 + ((uint32_t(c) ^ sw) << 4));
 #pragma unroll
   for (int c = 0; c < 8; ++c) {  // codes of columns 16c .. 16c + 15
-    const uint32_t words[4] = {w[c].x, w[c].y, w[c].z, w[c].w};
+    const uint4 w = *reinterpret_cast<const uint4*>(codes + r * 128 + ((uint32_t(c) ^ sw) << 4));
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
     uint32_t out[8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -540,8 +537,14 @@ __device__ __forceinline__ bool visible(uint32_t q0, uint32_t q1, uint32_t k, ui
 // attention forward
 // ---------------------------------------------------------------------------
 
-constexpr int kStages = 4;
-constexpr int kThreads = 384;     // 3 warpgroups
+constexpr int kStages = 4;       // bf16 cache: K/V ring depth (the most any instantiation uses)
+constexpr int kStagesInt8 = 3;   // INT8 cache: ring depth (room for the code slots)
+constexpr int kCodeSlots = 4;    // INT8 cache: staged code tiles
+__host__ __device__ constexpr int ring_stages(bool int8) { return int8 ? kStagesInt8 : kStages; }
+static_assert(kStagesInt8 <= kStages, "the barrier map holds kStages ring slots");
+constexpr int kThreads = 384;     // 3 warpgroups (bf16 cache)
+constexpr int kThreadsInt8 = 512; // + a dequantising warpgroup (INT8 cache)
+__host__ __device__ constexpr int threads_for(bool int8) { return int8 ? kThreadsInt8 : kThreads; }
 // Registers are split per warpgroup with setmaxnreg: the launch reserves
 // 384 x 168 = 64,512 (168 is the most a thread can get when three warps share
 // an SM sub-partition's 16K registers); the two softmax warpgroups grow to 224
@@ -551,6 +554,16 @@ constexpr int kRegsSoftmax = 224;
 constexpr int kRegsControl = 56;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl == kThreads * 168,
               "the register split must add up to the launch's registers");
+// INT8: 512 threads launch with 128 registers each; the softmax warpgroups
+// grow to 216 and the control and dequantising warpgroups shrink to 40
+// (2 x 128 x 216 + 2 x 128 x 40 = 512 x 128; the split ptxas fits without
+// spilling).
+constexpr int kRegsSoftmaxInt8 = 216;
+constexpr int kRegsControlInt8 = 40;
+constexpr int kRegsDequantInt8 = 40;
+static_assert(2 * 128 * kRegsSoftmaxInt8 + 128 * (kRegsControlInt8 + kRegsDequantInt8) ==
+                  kThreadsInt8 * 128,
+              "the INT8 register split must add up to the launch's registers");
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint32_t kHalf = 128 * 64 * 2;  // one 128-row x 64-column bf16 box: 16 KB
@@ -561,30 +574,42 @@ constexpr int kPolyEvery = 0;             // every n-th exponential pair of FULL
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr uint32_t kOffQ = 0;                            // Q0, Q1
 constexpr uint32_t kOffKV = 2 * kTile;                   // ring of K/V tiles
-// INT8 cache only: two staged code tiles (slot 0 takes the K tiles, slot 1
-// the V tiles) and their 128 row scales
+// INT8 cache only: kCodeSlots staged code tiles and their 128 row scales
 constexpr uint32_t kCodeTile = 128 * 128;                // 16 KB
-constexpr uint32_t kOffCodes = kOffKV + kStages * kTile;
-constexpr uint32_t kOffScales = kOffCodes + 2 * kCodeTile;
 constexpr uint32_t kScaleBytes = 128 * 4;
-__host__ __device__ constexpr uint32_t off_bar(bool int8) { return int8 ? kOffScales + 2 * kScaleBytes : kOffCodes; }
+__host__ __device__ constexpr uint32_t off_codes(bool int8) { return kOffKV + ring_stages(int8) * kTile; }
+__host__ __device__ constexpr uint32_t off_scales(bool int8) { return off_codes(int8) + kCodeSlots * kCodeTile; }
+__host__ __device__ constexpr uint32_t off_bar(bool int8) {
+  return int8 ? off_scales(int8) + kCodeSlots * kScaleBytes : off_codes(int8);
+}
 constexpr uint32_t kBarQ = 0, kBarFull = 1, kBarEmpty = kBarFull + kStages,
                    kBarS = kBarEmpty + kStages, kBarP = kBarS + 2, kBarO = kBarP + 2,
                    kBarDrain = kBarO + 2, kBarCodeFull = kBarDrain + 1,
-                   kBarCodeEmpty = kBarCodeFull + 2, kNumBars = kBarCodeEmpty + 2;
-__host__ __device__ constexpr uint32_t smem_bytes(bool int8) {
-  return off_bar(int8) + kNumBars * 8 + 16 + 16 + 1024;  // bars, control, TMEM slot, alignment slack
+                   kBarCodeEmpty = kBarCodeFull + kCodeSlots, kNumBars = kBarCodeEmpty + kCodeSlots;
+// The tiles need a 1024-byte aligned base. The dynamic shared window is
+// padded so that the base can be moved up to the next boundary: by a full
+// 1024 bytes when that fits the 227 KB a CTA may use (bf16), else by what is
+// left (INT8, whose 4 code slots leave about 800 bytes). CUDA places the
+// window on a 1024-byte boundary, so no padding is used in practice; a base
+// the padding cannot fix makes the kernel report SCA_ERR_MISALIGNED.
+constexpr uint32_t kSmemLimit = 232448;
+__host__ __device__ constexpr uint32_t smem_used(bool int8) {
+  return off_bar(int8) + kNumBars * 8 + 16 + 16;  // bars, control, TMEM slot
 }
-static_assert(smem_bytes(true) <= 232448, "the INT8 layout must fit the 227 KB a CTA may use");
+__host__ __device__ constexpr uint32_t align_slack(bool int8) {
+  return kSmemLimit - smem_used(int8) < 1024 ? kSmemLimit - smem_used(int8) : 1024;
+}
+__host__ __device__ constexpr uint32_t smem_bytes(bool int8) { return smem_used(int8) + align_slack(int8); }
+static_assert(smem_used(true) + 512 <= kSmemLimit, "the INT8 layout must fit the 227 KB a CTA may use");
 
 size_t attention_smem_bytes(bool int8_cache) { return smem_bytes(int8_cache); }
 
 // kInt8: the cache holds int8 codes with per-row scales (tm_kcache and
-// tm_vcache cover the codes, tm_kscale and tm_vscale the scales); the softmax
-// warpgroups dequantise the cache tiles into the operand ring one step ahead
-// of the MMAs. Otherwise the cache is bf16 and the scale maps are unused.
+// tm_vcache cover the codes, tm_kscale and tm_vscale the scales); a fourth
+// warpgroup dequantises the cache tiles into the operand ring ahead of the
+// MMAs. Otherwise the cache is bf16 and the scale maps are unused.
 template <bool kInt8>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_for(kInt8), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_kcur,
                     const __grid_constant__ CUtensorMap tm_vcur,
@@ -592,10 +617,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_vcache,
                     const __grid_constant__ CUtensorMap tm_kscale,
                     const __grid_constant__ CUtensorMap tm_vscale, const AttnArgs p) {
+  constexpr int kRing = ring_stages(kInt8);
+  constexpr uint32_t kOffCodes = off_codes(kInt8), kOffScales = off_scales(kInt8);
   constexpr uint32_t kOffBar = off_bar(kInt8);
   constexpr uint32_t kOffCtl = kOffBar + kNumBars * 8;
   constexpr uint32_t kOffTmemSlot = kOffCtl + 16;
   extern __shared__ uint8_t smem_raw[];
+  if ((1024u - (smem_u32(smem_raw) & 1023u)) % 1024u > align_slack(kInt8)) {
+    // the padding does not reach the next 1024-byte boundary: report
+    // instead of running misaligned (never taken with the full 1024)
+    if (threadIdx.x == 0 && p.status) atomicExch(p.status, SCA_ERR_MISALIGNED);
+    return;
+  }
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -627,12 +660,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     ctl->abort = 0;
     mbar_init(bar(kBarQ), 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kRing; ++s) {
       // INT8: a dequantised tile is complete after its warpgroup's 128 arrivals
       mbar_init(bar(kBarFull + s), kInt8 ? 128 : 1);
       mbar_init(bar(kBarEmpty + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kCodeSlots; ++s) {
       mbar_init(bar(kBarCodeFull + s), 1);
       mbar_init(bar(kBarCodeEmpty + s), 128);
     }
@@ -657,7 +690,30 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 8) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
+  if (kInt8 && warp >= 12) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsDequantInt8));
+    // ------------------------------------------------------------ dequantiser
+    // INT8 cache: thread r converts row r of every cache tile of the list (K
+    // and V alternate; the cache tiles are a prefix of the ascending list)
+    // from its staged code slot into the operand ring, as soon as the codes
+    // have landed and the ring slot is free.
+    const int r = int(threadIdx.x) - 384;
+    for (int it = 0; it < 2 * n_iter; ++it) {
+      if (int(list[it >> 1] & kPairTileMask) >= p.n_cache_tiles) break;
+      const int slot8 = it % kCodeSlots, s = it % kRing;
+      const bool ready = wait_bar(bar(kBarCodeFull + slot8), uint32_t(it / kCodeSlots) & 1u, ctl,
+                                  p.status, p.timeout_ns) &&
+                         wait_bar(bar(kBarEmpty + s), (uint32_t(it / kRing) & 1u) ^ 1u, ctl,
+                                  p.status, p.timeout_ns);
+      if (!__all_sync(0xFFFFFFFFu, ready)) break;
+      const float sc = reinterpret_cast<const float*>(smem + kOffScales + slot8 * kScaleBytes)[r];
+      dequant_row(smem + kOffCodes + slot8 * kCodeTile, sc, smem + kOffKV + s * kTile, r);
+      fence_proxy_async_smem();
+      mbar_arrive(bar(kBarFull + s));
+      mbar_arrive(bar(kBarCodeEmpty + slot8));
+    }
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kInt8 ? kRegsControlInt8 : kRegsControl));
   if (warp >= 10) {
     // warps 10-11 only complete the control warpgroup
   } else if (warp == kLoadWarp) {
@@ -678,21 +734,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tile = int(list[j] & kPairTileMask);
         for (int kv = 0; kv < 2; ++kv, ++it) {
           if (staged(it)) {
-            const uint32_t cb = bar(kBarCodeFull + kv);
-            if (!wait_bar(bar(kBarCodeEmpty + kv), (uint32_t(it >> 1) & 1u) ^ 1u, ctl, p.status,
-                          p.timeout_ns)) {
+            const int cs = it % kCodeSlots;
+            const uint32_t cb = bar(kBarCodeFull + cs);
+            if (!wait_bar(bar(kBarCodeEmpty + cs), (uint32_t(it / kCodeSlots) & 1u) ^ 1u, ctl,
+                          p.status, p.timeout_ns)) {
               ok = false;
               break;
             }
             mbar_expect_tx(cb, kCodeTile + kScaleBytes);
-            tma_load_3d(sbase + kOffCodes + uint32_t(kv) * kCodeTile, kv ? &tm_vcache : &tm_kcache,
+            tma_load_3d(sbase + kOffCodes + uint32_t(cs) * kCodeTile, kv ? &tm_vcache : &tm_kcache,
                         cb, 0, tile * 128, head);
-            tma_load_2d(sbase + kOffScales + uint32_t(kv) * kScaleBytes,
+            tma_load_2d(sbase + kOffScales + uint32_t(cs) * kScaleBytes,
                         kv ? &tm_vscale : &tm_kscale, cb, tile * 128, head);
             continue;
           }
-          const int s = it % kStages;
-          const uint32_t ph = uint32_t(it / kStages) & 1u;
+          if (kInt8 && it > 0 && staged(it - 1)) {
+            // first direct load after the staged prefix: wait until every
+            // staged tile is dequantised. Ring slots of the prefix were
+            // claimed by the dequantiser, so their release barriers may lag
+            // this thread's count by more than one phase, which a parity
+            // wait cannot tell apart; once the prefix is done they cannot.
+            for (int i2 = it - kCodeSlots < 0 ? 0 : it - kCodeSlots; i2 < it && ok; ++i2)
+              ok = wait_bar(bar(kBarCodeEmpty + i2 % kCodeSlots), uint32_t(i2 / kCodeSlots) & 1u, ctl,
+                            p.status, p.timeout_ns);
+            if (!ok) break;
+          }
+          const int s = it % kRing;
+          const uint32_t ph = uint32_t(it / kRing) & 1u;
           if (!wait_bar(bar(kBarEmpty + s), ph ^ 1u, ctl, p.status, p.timeout_ns)) {
             ok = false;
             break;
@@ -713,19 +781,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!ok) {
-        // drain: let every armed load land before the CTA can exit. A ring
-        // slot's latest load is among the last kStages issued; a code slot's
-        // is the last staged load of its parity (staged loads form a prefix).
-        for (int back = 1; back <= kStages && it - back >= 0; ++back) {
+        // drain: let every armed load land before the CTA can exit. The
+        // latest load of each ring slot is among the last kRing issued (the
+        // staged loads among them filled no ring slot); that of each code
+        // slot among the last kCodeSlots staged loads, which form a prefix.
+        for (int back = 1; back <= kRing && it - back >= 0; ++back) {
           const int i2 = it - back;
-          if (!staged(i2)) {
-            wait_bounded(bar(kBarFull + i2 % kStages), uint32_t(i2 / kStages) & 1u, ctl, nullptr,
+          if (!staged(i2))
+            wait_bounded(bar(kBarFull + i2 % kRing), uint32_t(i2 / kRing) & 1u, ctl, nullptr,
                          p.timeout_ns);
-          } else if (i2 + 2 >= it || !staged(i2 + 2)) {
-            wait_bounded(bar(kBarCodeFull + (i2 & 1)), uint32_t(i2 >> 1) & 1u, ctl, nullptr,
-                         p.timeout_ns);
-          }
         }
+        int n_staged = 0;
+        while (n_staged < it && staged(n_staged)) ++n_staged;
+        for (int i2 = n_staged - kCodeSlots < 0 ? 0 : n_staged - kCodeSlots; i2 < n_staged; ++i2)
+          wait_bounded(bar(kBarCodeFull + i2 % kCodeSlots), uint32_t(i2 / kCodeSlots) & 1u, ctl,
+                       nullptr, p.timeout_ns);
         wait_bounded(bar(kBarQ), 0, ctl, nullptr, p.timeout_ns);
       }
     }
@@ -740,9 +810,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_pv = [&](uint32_t tO, uint32_t tP, uint32_t sV, bool acc) {
         mma_pv8(tO, tP, desc_mnmajor(sV), kIdescPV, acc ? 1u : 0u);
       };
-      auto stage_of = [&](int it) { return sbase + kOffKV + uint32_t(it % kStages) * kTile; };
+      auto stage_of = [&](int it) { return sbase + kOffKV + uint32_t(it % kRing) * kTile; };
       auto wait_full = [&](int it) {
-        return wait_bar(bar(kBarFull + it % kStages), uint32_t(it / kStages) & 1u, ctl, p.status,
+        return wait_bar(bar(kBarFull + it % kRing), uint32_t(it / kRing) & 1u, ctl, p.status,
                         p.timeout_ns);
       };
       // a tile of the pair that sees nothing of key tile j gets neither its
@@ -782,11 +852,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           issue_pv(tO1, tS1, stage_of(itV), acc1);
           acc1 = true;
         }
-        mma_commit(bar(kBarEmpty + itV % kStages));
+        mma_commit(bar(kBarEmpty + itV % kRing));
         if (more) {
           if (live(j + 1, 1)) issue_qk(tS1, sQ1, stage_of(itK));
           mma_commit(bar(kBarS + 1));
-          mma_commit(bar(kBarEmpty + itK % kStages));
+          mma_commit(bar(kBarEmpty + itK % kRing));
         }
       }
       mma_commit(bar(kBarO + 0));
@@ -797,9 +867,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   }
+  }
   } else {
     // ------------------------------------------------------------ softmax
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kInt8 ? kRegsSoftmaxInt8 : kRegsSoftmax));
     const int t = warp >> 2;           // query tile of the pair
     const int wq = warp & 3;           // TMEM lane quadrant
     const int r = wq * 32 + lane;      // row in the tile
@@ -812,34 +883,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool o_init = false;  // O_t holds a P V result (else its TMEM is undefined)
     bool ok = true;
     const uint64_t scale2 = f2(p.scale_log2, p.scale_log2);
-    // INT8 cache: warpgroup 1 dequantises the K tiles (it = 2j) and
-    // warpgroup 0 the V tiles (it = 2j + 1) of the list's cache prefix, each
-    // thread one row, so that after the P of step j the K of step j + 2 and
-    // the V of step j + 1 are ready (both a step before the MMAs need them).
-    int conv_it = 1 - t;  // next tile this warpgroup dequantises
-    auto convert_upto = [&](int last) -> bool {
-      for (; conv_it <= last && conv_it < 2 * n_iter; conv_it += 2) {
-        if (int(list[conv_it >> 1] & kPairTileMask) >= p.n_cache_tiles) {
-          conv_it = 2 * n_iter;  // past the prefix: nothing left to convert
-          break;
-        }
-        const int slot8 = conv_it & 1, s = conv_it % kStages;
-        bool ready = wait_bar(bar(kBarCodeFull + slot8), uint32_t(conv_it >> 1) & 1u, ctl, p.status,
-                              p.timeout_ns) &&
-                     wait_bar(bar(kBarEmpty + s), (uint32_t(conv_it / kStages) & 1u) ^ 1u, ctl,
-                              p.status, p.timeout_ns);
-        if (!__all_sync(0xFFFFFFFFu, ready)) return false;
-        const float sc = reinterpret_cast<const float*>(smem + kOffScales + slot8 * kScaleBytes)[r];
-        dequant_row(smem + kOffCodes + slot8 * kCodeTile, sc, smem + kOffKV + s * kTile, r);
-        fence_proxy_async_smem();
-        mbar_arrive(bar(kBarFull + s));
-        mbar_arrive(bar(kBarCodeEmpty + slot8));
-      }
-      return true;
-    };
-    if (kInt8 && !convert_upto(1 + t)) ok = false;
     uint32_t e_next = n_iter > 0 ? list[0] : 0u;
-    for (int j = 0; ok && j < n_iter; ++j) {
+    for (int j = 0; j < n_iter; ++j) {
       const uint32_t e = e_next;
       if (j + 1 < n_iter) e_next = list[j + 1];   // prefetch the next schedule entry
       const int tile = int(e & kPairTileMask);
@@ -930,10 +975,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kBarP + t));
-      if (kInt8 && !convert_upto(2 * j + 3 + t)) {
-        ok = false;
-        break;
-      }
     }
     // ---------------------------------------------------------- epilogue
     if (ok && n_iter > 0) ok = wait_bar(bar(kBarO + t), 0, ctl, p.status, p.timeout_ns);
@@ -1016,7 +1057,7 @@ static cudaError_t launch_attention_t(const AttnMaps& maps, const AttnArgs& args
     if (dev < 31) configured_mask |= 1 << dev;
   }
   const unsigned grid = unsigned(args.n_full) + unsigned(args.n_split) * unsigned(args.chunks);
-  attn_fwd_kernel<kInt8><<<grid, kThreads, kSmem, stream>>>(
+  attn_fwd_kernel<kInt8><<<grid, threads_for(kInt8), kSmem, stream>>>(
       maps.q, maps.k_cur, maps.v_cur, maps.k_cache, maps.v_cache, maps.k_scale, maps.v_scale, args);
   return cudaGetLastError();
 }
