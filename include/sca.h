@@ -321,6 +321,39 @@ SCA_API int sca_action_causal_attn_fwd_static_ws(const sca_kv_cache* cache,
                                                  float softmax_scale, int32_t* dev_status,
                                                  void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Attention backward, for layouts without cached segments (the packed,
+ * FLOPs-balanced training batches of the picx.dev summary, "Methodology ›
+ * Training Infrastructure"; the pages print no backward pass, so its
+ * gradients are those of the forward above). Per head, over the visible
+ * pairs, with P the row softmax (recomputed from the forward's LSE):
+ *   dV = Pᵀ dO,  dP = dO Vᵀ,  D_i = Σ_d dO_id O_id,  dS = P ∘ (dP − D),
+ *   dQ = scale · dS K,  dK = scale · dSᵀ Q.
+ * Arguments:
+ *   md     : built and uploaded; no cached segments (SCA_ERR_UNSUPPORTED);
+ *            the same layout, window and dropped blocks as the forward;
+ *   q, k, v, o, d_o : bf16 token-major [n][heads][128], n = the metadata's
+ *            queries (= keys): the forward's inputs, its output and dO;
+ *   lse    : fp32 [heads][n], the forward's (natural log);
+ *   dq, dk, dv : bf16 [n][heads][128], written (not accumulated);
+ *   workspace, workspace_bytes : device scratch of at least
+ *            sca_attn_bwd_workspace_bytes (256-byte aligned; required:
+ *            SCA_ERR_CAPACITY otherwise); it receives D and LSE·log2(e);
+ *   dev_status, stream : as for the forward.
+ * Three kernels on the stream: D and LSE, dQ (query tiles over their key
+ * tiles), dK and dV (key tiles over the query tiles that see them); no
+ * atomics, so the result does not depend on scheduling. The call allocates
+ * nothing. A key no query sees gets dK = dV = 0. */
+SCA_API int sca_action_causal_attn_bwd(const sca_metadata* md, int32_t heads, const void* q,
+                                       const void* k, const void* v, const void* o,
+                                       const float* lse, const void* d_o, void* dq, void* dk,
+                                       void* dv, float softmax_scale, void* workspace,
+                                       uint64_t workspace_bytes, int32_t* dev_status,
+                                       void* stream);
+
+/* Workspace the backward needs: 2 · heads · round_up(n, 128) floats. */
+SCA_API int sca_attn_bwd_workspace_bytes(const sca_metadata* md, int32_t heads, uint64_t* bytes);
+
 /* Message of the calling thread's last failure ("" if none). */
 SCA_API const char* sca_last_error(void);
 

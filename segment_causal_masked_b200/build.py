@@ -18,7 +18,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsca.so")
-SOURCES = ["sca_host.cpp", "sca_kernels.cu", "sca_static_ws.cu"]
+SOURCES = ["sca_host.cpp", "sca_kernels.cu", "sca_bwd.cu", "sca_static_ws.cu"]
+HEADERS = ["sca_internal.h", "sca_ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -38,7 +39,7 @@ def _newer(target: str, deps) -> bool:
 
 def build(verbose: bool = False, force: bool = False) -> str:
     deps = [os.path.join(CSRC, s) for s in SOURCES]
-    deps += [os.path.join(CSRC, "sca_internal.h"), os.path.join(INCLUDE, "sca.h")]
+    deps += [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, "sca.h")]
     if not force and _newer(LIB, deps):
         return LIB
     cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",

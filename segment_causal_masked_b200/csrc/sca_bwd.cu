@@ -1,0 +1,680 @@
+// Attention backward of libsca for NVIDIA B200 (sm_100a): dQ, dK, dV of the
+// action-aware causal attention for layouts without cached segments (the
+// packed training batches of [picx.dev summary, Methodology › Training
+// Infrastructure]). Per head, with P the row softmax of the visible scores
+// (recomputed from the forward's LSE), D_i = Σ_d dO_id O_id and
+// dS = P ∘ (dO Vᵀ − D):  dV = Pᵀ dO,  dQ = scale · dS K,  dK = scale · dSᵀ Q.
+//
+// Three kernels, one stream:
+//   bwd_prep_kernel   D and LSE·log2(e) per (head, query) into the workspace;
+//   bwd_dq_kernel     one CTA per (query tile, head), over the query tile's
+//                     key tiles: S = Q Kᵀ and dP = dO Vᵀ into TMEM, dS in
+//                     registers, dQ += dS K accumulated in TMEM;
+//   bwd_dkdv_kernel   one CTA per (key tile, head), over the query tiles that
+//                     see it: Sᵀ = K Qᵀ and dPᵀ = V dOᵀ into TMEM, Pᵀ and dSᵀ
+//                     (bf16) back into TMEM, dV += Pᵀ dO and dK += dSᵀ Q.
+// S and dP are computed twice (once per kernel) so that neither dQ nor dK/dV
+// needs atomics. The schedules are the forward's tile classes: the dQ kernel
+// reads the pair work list, the dK/dV kernel its transpose (per key tile, the
+// query tiles with their classes); PARTIAL tiles are masked with the same
+// predicate on descriptor words, per run of equal descriptors.
+//
+// Warp roles (384 threads, as in the forward): warps 0-3 and 4-7 do the
+// elementwise work of columns 0-63 and 64-127 of every row (one thread per
+// TMEM lane, so no row needs a reduction: D and the LSE are precomputed);
+// warp 8 issues the TMA loads; warp 9 allocates TMEM and issues the MMAs.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sca_internal.h"
+#include "sca_ptx.cuh"
+
+namespace sca {
+
+namespace {
+
+constexpr int kBThreads = 384;
+constexpr int kBRegsWork = 224;
+constexpr int kBRegsControl = 56;
+static_assert(2 * 128 * kBRegsWork + 128 * kBRegsControl == kBThreads * 168,
+              "the register split must add up to the launch's registers");
+constexpr uint32_t kBHalf = 128 * 64 * 2;  // 128 rows x 64 bf16 columns
+constexpr uint32_t kBTile = 2 * kBHalf;    // 128 x 128 bf16
+constexpr float kLog2e = 1.4426950408889634f;
+
+// D (+)= A B with A from TMEM as two 32-column halves (keys or queries 0-63 at
+// a_lo, 64-127 at a_hi; 8 columns per K-step of 16) and B MN-major in shared
+// memory (2048 B per K-step). `acc` = 0 overwrites D on the first step.
+__device__ __forceinline__ void mma_ts8_split(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
+                                              uint64_t b_desc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred pf, pt;\n\t.reg .b32 ta, bl;\n\t.reg .b64 bd;\n\t"
+      "setp.ne.b32 pf, %6, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\t"
+      "mov.b64 bd, {%3, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %5, pf;\n\t"
+      "add.u32 ta, %1, 8;\n\tadd.u32 bl, %3, 128;\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %5, pt;\n\t"
+      "add.u32 ta, %1, 16;\n\tadd.u32 bl, %3, 256;\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %5, pt;\n\t"
+      "add.u32 ta, %1, 24;\n\tadd.u32 bl, %3, 384;\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %5, pt;\n\t"
+      "add.u32 bl, %3, 512;\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], bd, %5, pt;\n\t"
+      "add.u32 ta, %2, 8;\n\tadd.u32 bl, %3, 640;\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %5, pt;\n\t"
+      "add.u32 ta, %2, 16;\n\tadd.u32 bl, %3, 768;\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %5, pt;\n\t"
+      "add.u32 ta, %2, 24;\n\tadd.u32 bl, %3, 896;\n\tmov.b64 bd, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %5, pt;\n\t}"
+      ::"r"(d_tmem), "r"(a_lo), "r"(a_hi), "r"(uint32_t(b_desc)), "r"(uint32_t(b_desc >> 32)),
+      "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// Columns [c0, c0 + 64) of a run [a, b) as two 32-bit masks.
+__device__ __forceinline__ void set_run_bits(uint32_t (&vis)[2], int a, int b, int c0) {
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    const int lo = max(a, c0 + 32 * w) - (c0 + 32 * w);
+    const int hi = min(b, c0 + 32 * w + 32) - (c0 + 32 * w);
+    if (lo < hi) vis[w] |= uint32_t(((1ull << (hi - lo)) - 1ull) << lo);
+  }
+}
+
+// p = exp2(s * scale_log2 - l) where visible (0 elsewhere), ds = p (dp - d);
+// 64 columns -> 32 bf16 pairs of p and of ds.
+__device__ __forceinline__ void p_ds_row(const float (&s)[64], const float (&dp)[64],
+                                         const uint32_t (&vis)[2], bool full, float scale_log2,
+                                         float l, float d, uint32_t (&pw)[32], uint32_t (&dsw)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    float p0 = ex2(fmaf(s[2 * i], scale_log2, -l));
+    float p1 = ex2(fmaf(s[2 * i + 1], scale_log2, -l));
+    if (!full) {
+      p0 = ((vis[(2 * i) >> 5] >> ((2 * i) & 31)) & 1u) ? p0 : 0.f;
+      p1 = ((vis[(2 * i + 1) >> 5] >> ((2 * i + 1) & 31)) & 1u) ? p1 : 0.f;
+    }
+    pw[i] = pack_bf16(p0, p1);
+    dsw[i] = pack_bf16(p0 * (dp[2 * i] - d), p1 * (dp[2 * i + 1] - d));
+  }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// D = rowsum(dO ∘ O) and LSE · log2(e), per (head, query)
+// ---------------------------------------------------------------------------
+
+// One warp per (query, head) row, 4 values per lane. Rows past n (up to the
+// tile-padded n_pad) get D = 0 and L = 0; the kernels never use them
+// unmasked. A row with LSE = -inf (it sees nothing) gets L = +inf, so that
+// its probabilities come out 0.
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
+  const uint2* __restrict__ o = static_cast<const uint2*>(a.o);
+  const uint2* __restrict__ g = static_cast<const uint2*>(a.d_o);
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = int64_t(a.n_pad) * a.heads;
+  const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t row = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); row < rows;
+       row += wstride) {
+    const int64_t tok = row / a.heads;
+    const int h = int(row - tok * a.heads);
+    float d = 0.f, l = 0.f;
+    if (tok < a.n) {
+      const uint2 x = __ldg(o + row * 32 + lane);
+      const uint2 y = __ldg(g + row * 32 + lane);
+      d = __uint_as_float(x.x << 16) * __uint_as_float(y.x << 16) +
+          __uint_as_float(x.x & 0xFFFF0000u) * __uint_as_float(y.x & 0xFFFF0000u) +
+          __uint_as_float(x.y << 16) * __uint_as_float(y.y << 16) +
+          __uint_as_float(x.y & 0xFFFF0000u) * __uint_as_float(y.y & 0xFFFF0000u);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) d += __shfl_xor_sync(0xFFFFFFFFu, d, off);
+      const float lse = a.lse[int64_t(h) * a.n + tok];
+      l = lse == -INFINITY ? INFINITY : lse * kLog2e;
+    }
+    if (lane == 0) {
+      a.dl[int64_t(h) * a.n_pad + tok] = d;
+      a.dl[int64_t(a.heads + h) * a.n_pad + tok] = l;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dQ
+// ---------------------------------------------------------------------------
+
+// shared memory (1024-aligned base): Q, dO, a ring of 3 K tiles and one of 2
+// V tiles (K_j is read by S_j and, a step later, by dQ += dS_j K_j).
+constexpr uint32_t kQOffQ = 0, kQOffDO = kBTile, kQOffK = 2 * kBTile, kQOffV = 5 * kBTile;
+constexpr int kQKSlots = 3, kQVSlots = 2;
+constexpr uint32_t kQBarQD = 0, kQBarKF = 1, kQBarKE = kQBarKF + kQKSlots,
+                   kQBarVF = kQBarKE + kQKSlots, kQBarVE = kQBarVF + kQVSlots,
+                   kQBarS = kQBarVE + kQVSlots, kQBarDP = kQBarS + 2, kQBarDS = kQBarDP + 1,
+                   kQBarDone = kQBarDS + 1, kQBarDrain = kQBarDone + 1, kQNumBars = kQBarDrain + 1;
+constexpr uint32_t kQOffBar = 7 * kBTile;
+constexpr uint32_t kQOffCtl = kQOffBar + kQNumBars * 8;
+constexpr uint32_t kQOffSlot = kQOffCtl + 16;
+constexpr uint32_t kQSmem = kQOffSlot + 16 + 1024;
+static_assert(kQSmem <= 232448, "the dQ kernel must fit the 227 KB a CTA may use");
+
+__global__ void __launch_bounds__(kBThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_do, const BwdArgs p) {
+  const int head = int(blockIdx.x) % p.heads;
+  const int rest = int(blockIdx.x) / p.heads;
+  const int t = rest & 1;                        // which tile of the pair
+  const int pair = p.item_order[rest >> 1];
+  const int qtile = 2 * pair + t;
+  if (qtile >= p.n_q_tiles) return;              // the odd last pair has one tile
+  const uint32_t* list = p.pair_list + p.pair_ptr[pair];
+  const int len = p.pair_ptr[pair + 1] - p.pair_ptr[pair];
+  auto cls_of = [&](int e) { return (list[e] >> (24 + 2 * t)) & 3u; };
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](uint32_t i) { return sbase + kQOffBar + 8 * i; };
+  volatile Ctl* ctl = reinterpret_cast<volatile Ctl*>(smem + kQOffCtl);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kQOffSlot);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    ctl->abort = 0;
+    mbar_init(bar(kQBarQD), 1);
+    for (int s = 0; s < kQKSlots; ++s) {
+      mbar_init(bar(kQBarKF + s), 1);
+      mbar_init(bar(kQBarKE + s), 1);
+    }
+    for (int s = 0; s < kQVSlots; ++s) {
+      mbar_init(bar(kQBarVF + s), 1);
+      mbar_init(bar(kQBarVE + s), 1);
+    }
+    mbar_init(bar(kQBarS), 1);
+    mbar_init(bar(kQBarS + 1), 1);
+    mbar_init(bar(kQBarDP), 1);
+    mbar_init(bar(kQBarDS), 256);
+    mbar_init(bar(kQBarDone), 1);
+    mbar_init(bar(kQBarDrain), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 9) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     smem_u32(tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS0 = tmem, tDP = tmem + 256, tDQ = tmem + 384;
+
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kBRegsControl));
+    if (warp == 8 && lane == 0) {
+      // ---------------------------------------------------------------- producer
+      mbar_expect_tx(bar(kQBarQD), 2 * kBTile);
+      const int q0 = qtile * 128;
+      tma_load_3d(sbase + kQOffQ, &tm_q, bar(kQBarQD), 0, head, q0);
+      tma_load_3d(sbase + kQOffQ + kBHalf, &tm_q, bar(kQBarQD), 64, head, q0);
+      tma_load_3d(sbase + kQOffDO, &tm_do, bar(kQBarQD), 0, head, q0);
+      tma_load_3d(sbase + kQOffDO + kBHalf, &tm_do, bar(kQBarQD), 64, head, q0);
+      int j = 0;
+      bool ok = true;
+      for (int e = 0; e < len && ok; ++e) {
+        if (cls_of(e) == SCA_TILE_EMPTY) continue;
+        const int row = int(list[e] & kPairTileMask) * 128;
+        const int ks = j % kQKSlots, vs = j % kQVSlots;
+        ok = wait_bar(bar(kQBarKE + ks), (uint32_t(j / kQKSlots) & 1u) ^ 1u, ctl, p.status,
+                      p.timeout_ns);
+        if (!ok) break;
+        mbar_expect_tx(bar(kQBarKF + ks), kBTile);
+        tma_load_3d(sbase + kQOffK + ks * kBTile, &tm_k, bar(kQBarKF + ks), 0, head, row);
+        tma_load_3d(sbase + kQOffK + ks * kBTile + kBHalf, &tm_k, bar(kQBarKF + ks), 64, head, row);
+        ok = wait_bar(bar(kQBarVE + vs), (uint32_t(j / kQVSlots) & 1u) ^ 1u, ctl, p.status,
+                      p.timeout_ns);
+        if (!ok) {
+          wait_bounded(bar(kQBarKF + ks), uint32_t(j / kQKSlots) & 1u, ctl, nullptr, p.timeout_ns);
+          break;
+        }
+        mbar_expect_tx(bar(kQBarVF + vs), kBTile);
+        tma_load_3d(sbase + kQOffV + vs * kBTile, &tm_v, bar(kQBarVF + vs), 0, head, row);
+        tma_load_3d(sbase + kQOffV + vs * kBTile + kBHalf, &tm_v, bar(kQBarVF + vs), 64, head, row);
+        ++j;
+      }
+      if (!ok) {
+        // drain: every armed load lands before the CTA can exit (the latest
+        // load of each slot is among the last kQKSlots / kQVSlots)
+        for (int i = j - kQKSlots < 0 ? 0 : j - kQKSlots; i < j; ++i)
+          wait_bounded(bar(kQBarKF + i % kQKSlots), uint32_t(i / kQKSlots) & 1u, ctl, nullptr,
+                       p.timeout_ns);
+        for (int i = j - kQVSlots < 0 ? 0 : j - kQVSlots; i < j; ++i)
+          wait_bounded(bar(kQBarVF + i % kQVSlots), uint32_t(i / kQVSlots) & 1u, ctl, nullptr,
+                       p.timeout_ns);
+        wait_bounded(bar(kQBarQD), 0, ctl, nullptr, p.timeout_ns);
+      }
+    } else if (warp == 9) {
+      // ---------------------------------------------------------------- MMA
+      int n = 0;  // live key tiles of this query tile, counted by the warp
+      for (int e0 = 0; e0 < len; e0 += 32) {
+        const bool live = e0 + lane < len && cls_of(e0 + lane) != SCA_TILE_EMPTY;
+        n += __popc(__ballot_sync(0xFFFFFFFFu, live));
+      }
+      if (lane == 0) {
+        const uint64_t dQ = desc_kmajor(sbase + kQOffQ), dDO = desc_kmajor(sbase + kQOffDO);
+        auto kslot = [&](int j) { return sbase + kQOffK + uint32_t(j % kQKSlots) * kBTile; };
+        auto vslot = [&](int j) { return sbase + kQOffV + uint32_t(j % kQVSlots) * kBTile; };
+        auto wait_k = [&](int j) {
+          return wait_bar(bar(kQBarKF + j % kQKSlots), uint32_t(j / kQKSlots) & 1u, ctl, p.status,
+                          p.timeout_ns);
+        };
+        auto wait_v = [&](int j) {
+          return wait_bar(bar(kQBarVF + j % kQVSlots), uint32_t(j / kQVSlots) & 1u, ctl, p.status,
+                          p.timeout_ns);
+        };
+        // Q and dO are always loaded: wait for them even with no key tile
+        bool ok = wait_bar(bar(kQBarQD), 0, ctl, p.status, p.timeout_ns);
+        if (ok && n > 0) {
+          ok = wait_k(0);
+          if (ok) {
+            tc_fence_after();
+            mma_qk8(tS0, dQ, desc_kmajor(kslot(0)), kIdescQK);
+            mma_commit(bar(kQBarS));
+            ok = wait_v(0);
+          }
+          if (ok) {
+            tc_fence_after();
+            mma_qk8(tDP, dDO, desc_kmajor(vslot(0)), kIdescQK);
+            mma_commit(bar(kQBarDP));
+            mma_commit(bar(kQBarVE));
+          }
+          if (ok && n > 1 && (ok = wait_k(1))) {
+            tc_fence_after();
+            mma_qk8(tS0 + 128, dQ, desc_kmajor(kslot(1)), kIdescQK);
+            mma_commit(bar(kQBarS + 1));
+          }
+        }
+        for (int j = 0; ok && j < n; ++j) {
+          const uint32_t tSj = tS0 + uint32_t(j & 1) * 128;
+          if (!(ok = wait_bar(bar(kQBarDS), uint32_t(j) & 1u, ctl, p.status, p.timeout_ns))) break;
+          tc_fence_after();
+          if (j + 1 < n) {  // dP of the next key tile first: the elementwise warps wait on it
+            if (!(ok = wait_v(j + 1))) break;
+            tc_fence_after();
+            mma_qk8(tDP, dDO, desc_kmajor(vslot(j + 1)), kIdescQK);
+            mma_commit(bar(kQBarDP));
+            mma_commit(bar(kQBarVE + (j + 1) % kQVSlots));
+          }
+          mma_ts8_split(tDQ, tSj, tSj + 64, desc_mnmajor(kslot(j)), kIdescPV, j > 0 ? 1u : 0u);
+          mma_commit(bar(kQBarKE + j % kQKSlots));
+          if (j + 2 < n) {  // S of the key tile after next into the slot dS_j leaves
+            if (!(ok = wait_k(j + 2))) break;
+            tc_fence_after();
+            mma_qk8(tSj, dQ, desc_kmajor(kslot(j + 2)), kIdescQK);
+            mma_commit(bar(kQBarS + (j & 1)));
+          }
+        }
+        mma_commit(bar(kQBarDone));
+        mma_commit(bar(kQBarDrain));
+        wait_bounded(bar(kQBarDrain), 0, ctl, nullptr, p.timeout_ns);
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------------------------ elementwise
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kBRegsWork));
+    const int half = warp >> 2;                   // columns [64 half, 64 half + 64)
+    const int r = (warp & 3) * 32 + lane;         // row = TMEM lane
+    const int q_row = qtile * 128 + r;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint2 qd = p.qdesc[q_row];
+    const float l = p.dl[int64_t(p.heads + head) * p.n_pad + q_row];
+    const float d = p.dl[int64_t(head) * p.n_pad + q_row];
+    const int c0 = 64 * half;
+    bool ok = true;
+    int j = 0;
+    for (int e = 0; e < len; ++e) {
+      const uint32_t cls = cls_of(e);
+      if (cls == SCA_TILE_EMPTY) continue;
+      const int tile = int(list[e] & kPairTileMask);
+      uint32_t vis[2] = {0u, 0u};
+      if (cls == SCA_TILE_PARTIAL) {
+        for (int i = p.run_ptr[tile]; i < p.run_ptr[tile + 1]; ++i) {
+          const uint2 run = p.runs[i];
+          if (!visible(qd.x, qd.y, run.y, uint32_t(p.history))) continue;
+          const int a = int(run.x & 255u);
+          set_run_bits(vis, a, a + int((run.x >> 8) & 255u), c0);
+        }
+      }
+      ok = wait_bar(bar(kQBarS + (j & 1)), uint32_t(j >> 1) & 1u, ctl, p.status, p.timeout_ns) &&
+           wait_bar(bar(kQBarDP), uint32_t(j) & 1u, ctl, p.status, p.timeout_ns);
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tSj = tS0 + uint32_t(j & 1) * 128 + lane_base;
+      float s[64], dp[64];
+      tmem_ld32(tSj + c0, s);
+      tmem_ld32(tSj + c0 + 32, s + 32);
+      tmem_ld32(tDP + lane_base + c0, dp);
+      tmem_ld32(tDP + lane_base + c0 + 32, dp + 32);
+      tmem_wait_ld();
+      uint32_t pw[32], dsw[32];
+      p_ds_row(s, dp, vis, cls == SCA_TILE_FULL, p.scale_log2, l, d, pw, dsw);
+      tmem_st16(tSj + c0, dsw);  // dS over the first 32 columns of this half
+      tmem_st16(tSj + c0 + 16, dsw + 16);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kQBarDS));
+      ++j;
+    }
+    // epilogue: dQ row (this half) = scale * accumulated dS K
+    if (ok) ok = wait_bar(bar(kQBarDone), 0, ctl, p.status, p.timeout_ns);
+    if (__all_sync(0xFFFFFFFFu, ok)) {
+      tc_fence_after();
+      float g[64];
+      if (j > 0) {
+        tmem_ld32(tDQ + lane_base + c0, g);
+        tmem_ld32(tDQ + lane_base + c0 + 32, g + 32);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) g[i] = 0.f;
+      }
+      if (q_row < p.n) {
+        uint4* out = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dq) +
+                                              (int64_t(q_row) * p.heads + head) * 128 + c0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          out[i] = make_uint4(pack_bf16(g[8 * i] * p.scale, g[8 * i + 1] * p.scale),
+                              pack_bf16(g[8 * i + 2] * p.scale, g[8 * i + 3] * p.scale),
+                              pack_bf16(g[8 * i + 4] * p.scale, g[8 * i + 5] * p.scale),
+                              pack_bf16(g[8 * i + 6] * p.scale, g[8 * i + 7] * p.scale));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dK and dV
+// ---------------------------------------------------------------------------
+
+// shared memory: K, V of the CTA's key tile, then 2 stages of (Q, dO, D, L)
+// of one query tile (65 KB each, so every tile stays 1024-aligned).
+constexpr uint32_t kKOffK = 0, kKOffV = kBTile, kKOffStage = 2 * kBTile;
+constexpr uint32_t kKStage = 2 * kBTile + 1024;  // Q, dO, D[128], L[128]
+constexpr int kKStages = 2;
+constexpr uint32_t kKBarKV = 0, kKBarF = 1, kKBarE = kKBarF + kKStages, kKBarSDP = kKBarE + kKStages,
+                   kKBarDS = kKBarSDP + 1, kKBarDone = kKBarDS + 1, kKBarDrain = kKBarDone + 1,
+                   kKNumBars = kKBarDrain + 1;
+constexpr uint32_t kKOffBar = kKOffStage + kKStages * kKStage;
+constexpr uint32_t kKOffCtl = kKOffBar + kKNumBars * 8;
+constexpr uint32_t kKOffSlot = kKOffCtl + 16;
+constexpr uint32_t kKSmem = kKOffSlot + 16 + 1024;
+static_assert(kKSmem <= 232448, "the dK/dV kernel must fit the 227 KB a CTA may use");
+static_assert(kKStage % 1024 == 0, "stages must keep the tiles 1024-aligned");
+
+__global__ void __launch_bounds__(kBThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_dl, const BwdArgs p) {
+  const int head = int(blockIdx.x) % p.heads;
+  const int ktile = p.kt_order[int(blockIdx.x) / p.heads];
+  const uint32_t* list = p.kt_list + p.kt_ptr[ktile];
+  const int n = p.kt_ptr[ktile + 1] - p.kt_ptr[ktile];
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto bar = [&](uint32_t i) { return sbase + kKOffBar + 8 * i; };
+  auto stage = [&](int i) { return kKOffStage + uint32_t(i % kKStages) * kKStage; };
+  volatile Ctl* ctl = reinterpret_cast<volatile Ctl*>(smem + kKOffCtl);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kKOffSlot);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    ctl->abort = 0;
+    mbar_init(bar(kKBarKV), 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(bar(kKBarF + s), 1);
+      mbar_init(bar(kKBarE + s), 1);
+    }
+    mbar_init(bar(kKBarSDP), 1);
+    mbar_init(bar(kKBarDS), 256);
+    mbar_init(bar(kKBarDone), 1);
+    mbar_init(bar(kKBarDrain), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 9) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     smem_u32(tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tSt = tmem, tDPt = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
+
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kBRegsControl));
+    if (warp == 8 && lane == 0) {
+      // ---------------------------------------------------------------- producer
+      const int k0 = ktile * 128;
+      mbar_expect_tx(bar(kKBarKV), 2 * kBTile);
+      tma_load_3d(sbase + kKOffK, &tm_k, bar(kKBarKV), 0, head, k0);
+      tma_load_3d(sbase + kKOffK + kBHalf, &tm_k, bar(kKBarKV), 64, head, k0);
+      tma_load_3d(sbase + kKOffV, &tm_v, bar(kKBarKV), 0, head, k0);
+      tma_load_3d(sbase + kKOffV + kBHalf, &tm_v, bar(kKBarKV), 64, head, k0);
+      int i = 0;
+      bool ok = true;
+      for (; i < n; ++i) {
+        const int s = i % kKStages;
+        if (!(ok = wait_bar(bar(kKBarE + s), (uint32_t(i / kKStages) & 1u) ^ 1u, ctl, p.status,
+                            p.timeout_ns)))
+          break;
+        const int q0 = int(list[i] & kPairTileMask) * 128;
+        const uint32_t st = sbase + stage(i), fb = bar(kKBarF + s);
+        mbar_expect_tx(fb, 2 * kBTile + 1024);
+        tma_load_3d(st, &tm_q, fb, 0, head, q0);
+        tma_load_3d(st + kBHalf, &tm_q, fb, 64, head, q0);
+        tma_load_3d(st + kBTile, &tm_do, fb, 0, head, q0);
+        tma_load_3d(st + kBTile + kBHalf, &tm_do, fb, 64, head, q0);
+        tma_load_2d(st + 2 * kBTile, &tm_dl, fb, q0, head);
+        tma_load_2d(st + 2 * kBTile + 512, &tm_dl, fb, q0, p.heads + head);
+      }
+      if (!ok) {
+        for (int i2 = i - kKStages < 0 ? 0 : i - kKStages; i2 < i; ++i2)
+          wait_bounded(bar(kKBarF + i2 % kKStages), uint32_t(i2 / kKStages) & 1u, ctl, nullptr,
+                       p.timeout_ns);
+        wait_bounded(bar(kKBarKV), 0, ctl, nullptr, p.timeout_ns);
+      }
+    } else if (warp == 9 && lane == 0) {
+      // ---------------------------------------------------------------- MMA
+      const uint64_t dK = desc_kmajor(sbase + kKOffK), dV = desc_kmajor(sbase + kKOffV);
+      auto wait_f = [&](int i) {
+        return wait_bar(bar(kKBarF + i % kKStages), uint32_t(i / kKStages) & 1u, ctl, p.status,
+                        p.timeout_ns);
+      };
+      auto issue_sdp = [&](int i) {  // Sᵀ = K Qᵢᵀ, dPᵀ = V dOᵢᵀ
+        const uint32_t st = sbase + stage(i);
+        mma_qk8(tSt, dK, desc_kmajor(st), kIdescQK);
+        mma_qk8(tDPt, dV, desc_kmajor(st + kBTile), kIdescQK);
+        mma_commit(bar(kKBarSDP));
+      };
+      // K and V are always loaded: wait for them even with no query tile
+      bool ok = wait_bar(bar(kKBarKV), 0, ctl, p.status, p.timeout_ns) && (n == 0 || wait_f(0));
+      if (ok && n > 0) {
+        tc_fence_after();
+        issue_sdp(0);
+      }
+      for (int i = 0; ok && i < n; ++i) {
+        if (!(ok = wait_bar(bar(kKBarDS), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns))) break;
+        tc_fence_after();
+        const uint32_t st = sbase + stage(i);
+        // dV += Pᵀ dO, dK += dSᵀ Q (B MN-major: rows are queries)
+        mma_ts8_split(tDV, tSt, tSt + 64, desc_mnmajor(st + kBTile), kIdescPV, i > 0 ? 1u : 0u);
+        mma_ts8_split(tDK, tDPt, tDPt + 64, desc_mnmajor(st), kIdescPV, i > 0 ? 1u : 0u);
+        mma_commit(bar(kKBarE + i % kKStages));
+        if (i + 1 < n) {
+          if (!(ok = wait_f(i + 1))) break;
+          tc_fence_after();
+          issue_sdp(i + 1);
+        }
+      }
+      mma_commit(bar(kKBarDone));
+      mma_commit(bar(kKBarDrain));
+      wait_bounded(bar(kKBarDrain), 0, ctl, nullptr, p.timeout_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ elementwise
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kBRegsWork));
+    const int half = warp >> 2;                   // query columns [64 half, 64 half + 64)
+    const int r = (warp & 3) * 32 + lane;         // key row = TMEM lane
+    const int key = ktile * 128 + r;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t kd = p.kdesc[key];
+    const int c0 = 64 * half;
+    bool ok = true;
+    int i = 0;
+    for (; i < n; ++i) {
+      const uint32_t e = list[i];
+      const int qt = int(e & kPairTileMask);
+      const uint32_t cls = e >> 24;
+      uint32_t vis[2] = {0u, 0u};
+      if (cls == SCA_TILE_PARTIAL && key < p.n) {  // a padding key sees nothing
+        for (int k = p.qrun_ptr[qt]; k < p.qrun_ptr[qt + 1]; ++k) {
+          const uint4 run = p.qruns[k];
+          if (!visible(run.y, run.z, kd, uint32_t(p.history))) continue;
+          const int a = int(run.x & 255u);
+          set_run_bits(vis, a, a + int((run.x >> 8) & 255u), c0);
+        }
+      }
+      ok = wait_bar(bar(kKBarF + i % kKStages), uint32_t(i / kKStages) & 1u, ctl, p.status,
+                    p.timeout_ns) &&
+           wait_bar(bar(kKBarSDP), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns);
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[64], dp[64];
+      tmem_ld32(tSt + lane_base + c0, s);
+      tmem_ld32(tSt + lane_base + c0 + 32, s + 32);
+      tmem_ld32(tDPt + lane_base + c0, dp);
+      tmem_ld32(tDPt + lane_base + c0 + 32, dp + 32);
+      const float* dl = reinterpret_cast<const float*>(smem + stage(i) + 2 * kBTile);
+      tmem_wait_ld();
+      uint32_t pw[32], dsw[32];
+#pragma unroll
+      for (int c = 0; c < 64; c += 4) {  // per column: this query's D and L
+        const float4 dd = *reinterpret_cast<const float4*>(dl + c0 + c);
+        const float4 ll = *reinterpret_cast<const float4*>(dl + 128 + c0 + c);
+        const float dv4[4] = {dd.x, dd.y, dd.z, dd.w}, lv4[4] = {ll.x, ll.y, ll.z, ll.w};
+#pragma unroll
+        for (int u = 0; u < 4; u += 2) {
+          const int cc = c + u;
+          float p0 = ex2(fmaf(s[cc], p.scale_log2, -lv4[u]));
+          float p1 = ex2(fmaf(s[cc + 1], p.scale_log2, -lv4[u + 1]));
+          if (cls != SCA_TILE_FULL) {
+            p0 = ((vis[cc >> 5] >> (cc & 31)) & 1u) ? p0 : 0.f;
+            p1 = ((vis[(cc + 1) >> 5] >> ((cc + 1) & 31)) & 1u) ? p1 : 0.f;
+          }
+          pw[cc >> 1] = pack_bf16(p0, p1);
+          dsw[cc >> 1] = pack_bf16(p0 * (dp[cc] - dv4[u]), p1 * (dp[cc + 1] - dv4[u + 1]));
+        }
+      }
+      tmem_st16(tSt + lane_base + c0, pw);  // Pᵀ over the first 32 columns of this half
+      tmem_st16(tSt + lane_base + c0 + 16, pw + 16);
+      tmem_st16(tDPt + lane_base + c0, dsw);  // dSᵀ likewise
+      tmem_st16(tDPt + lane_base + c0 + 16, dsw + 16);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kKBarDS));
+    }
+    // epilogue: dV and dK rows (this half)
+    if (ok) ok = wait_bar(bar(kKBarDone), 0, ctl, p.status, p.timeout_ns);
+    if (__all_sync(0xFFFFFFFFu, ok)) {
+      tc_fence_after();
+      float gv[64], gk[64];
+      if (n > 0) {
+        tmem_ld32(tDV + lane_base + c0, gv);
+        tmem_ld32(tDV + lane_base + c0 + 32, gv + 32);
+        tmem_ld32(tDK + lane_base + c0, gk);
+        tmem_ld32(tDK + lane_base + c0 + 32, gk + 32);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) gv[c] = gk[c] = 0.f;
+      }
+      if (key < p.n) {
+        const int64_t off = (int64_t(key) * p.heads + head) * 128 + c0;
+        uint4* ov = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv) + off);
+        uint4* ok4 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk) + off);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          ov[c] = make_uint4(pack_bf16(gv[8 * c], gv[8 * c + 1]), pack_bf16(gv[8 * c + 2], gv[8 * c + 3]),
+                             pack_bf16(gv[8 * c + 4], gv[8 * c + 5]), pack_bf16(gv[8 * c + 6], gv[8 * c + 7]));
+          ok4[c] = make_uint4(pack_bf16(gk[8 * c] * p.scale, gk[8 * c + 1] * p.scale),
+                              pack_bf16(gk[8 * c + 2] * p.scale, gk[8 * c + 3] * p.scale),
+                              pack_bf16(gk[8 * c + 4] * p.scale, gk[8 * c + 5] * p.scale),
+                              pack_bf16(gk[8 * c + 6] * p.scale, gk[8 * c + 7] * p.scale));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+cudaError_t launch_backward(const BwdMaps& maps, const BwdArgs& args, cudaStream_t stream) {
+  static int configured_mask = 0;
+  int dev = 0, sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 31 || !(configured_mask & (1 << dev))) {
+    e = cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kQSmem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(kKSmem));
+    if (e != cudaSuccess) return e;
+    if (dev < 31) configured_mask |= 1 << dev;
+  }
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t rows = int64_t(args.n_pad) * args.heads;
+  int64_t blocks = (rows + 7) / 8;
+  blocks = blocks < int64_t(sms) * 16 ? blocks : int64_t(sms) * 16;
+  bwd_prep_kernel<<<unsigned(blocks), 256, 0, stream>>>(args);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  bwd_dq_kernel<<<unsigned(args.n_pairs * 2 * args.heads), kBThreads, kQSmem, stream>>>(
+      maps.q, maps.k, maps.v, maps.d_o, args);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  bwd_dkdv_kernel<<<unsigned(args.n_q_tiles * args.heads), kBThreads, kKSmem, stream>>>(
+      maps.q, maps.k, maps.v, maps.d_o, maps.dl, args);
+  return cudaGetLastError();
+}
+
+}  // namespace sca

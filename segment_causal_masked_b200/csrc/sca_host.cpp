@@ -387,6 +387,52 @@ int sca_build_segment_mask_metadata_ex(sca_metadata* md, const sca_segment* cach
     return pair_cost[size_t(x)] > pair_cost[size_t(y)];
   });
 
+  // --- backward work lists (layouts without a cache: keys = queries) ------
+  // per key tile, the query tiles that see it (the transposed schedule),
+  // longest list first; per query tile, runs of equal query descriptors; the
+  // key descriptors padded to whole tiles.
+  std::vector<int32_t> kt_ptr, kt_order, qrun_ptr;
+  std::vector<uint32_t> kt_list, qruns, kdesc_pad;
+  if (n_cached == 0) {
+    const int n_kt = int(n_ut);
+    kt_ptr.assign(size_t(n_kt) + 1, 0);
+    for (int32_t t : kv_tile) kt_ptr[size_t(t - n_ct) + 1] += 1;
+    for (int t = 0; t < n_kt; ++t) kt_ptr[size_t(t) + 1] += kt_ptr[size_t(t)];
+    kt_list.resize(kv_tile.size());
+    std::vector<int32_t> pos(kt_ptr.begin(), kt_ptr.end() - 1);
+    for (int qt = 0; qt < n_qt; ++qt)
+      for (int32_t i = row_ptr[size_t(qt)]; i < row_ptr[size_t(qt) + 1]; ++i)
+        kt_list[size_t(pos[size_t(kv_tile[size_t(i)] - n_ct)]++)] =
+            uint32_t(qt) | (uint32_t(flag[size_t(i)]) << 24);
+    std::vector<float> kt_cost(size_t(n_kt), 0.f);
+    for (int t = 0; t < n_kt; ++t)
+      for (int32_t i = kt_ptr[size_t(t)]; i < kt_ptr[size_t(t) + 1]; ++i)
+        kt_cost[size_t(t)] += w_cls[(kt_list[size_t(i)] >> 24) & 3u];
+    kt_order.resize(size_t(n_kt));
+    std::iota(kt_order.begin(), kt_order.end(), 0);
+    std::stable_sort(kt_order.begin(), kt_order.end(), [&](int32_t x, int32_t y) {
+      return kt_cost[size_t(x)] > kt_cost[size_t(y)];
+    });
+    qrun_ptr.assign(size_t(n_qt) + 1, 0);
+    for (int qt = 0; qt < n_qt; ++qt) {
+      const int64_t r0 = int64_t(qt) * SCA_TILE, r1 = std::min<int64_t>(n_q, r0 + SCA_TILE);
+      for (int64_t a = r0; a < r1;) {
+        int64_t b = a + 1;
+        while (b < r1 && qdesc[size_t(2 * b)] == qdesc[size_t(2 * a)] &&
+               qdesc[size_t(2 * b + 1)] == qdesc[size_t(2 * a + 1)])
+          ++b;
+        qruns.push_back(uint32_t(a - r0) | (uint32_t(b - a) << 8));
+        qruns.push_back(qdesc[size_t(2 * a)]);
+        qruns.push_back(qdesc[size_t(2 * a + 1)]);
+        qruns.push_back(0u);
+        a = b;
+      }
+      qrun_ptr[size_t(qt) + 1] = int32_t(qruns.size() / 4);
+    }
+    kdesc_pad.assign(size_t(n_qt) * SCA_TILE, 0u);
+    std::copy(kdesc_cur.begin(), kdesc_cur.end(), kdesc_pad.begin());
+  }
+
   md->built = true;
   md->uploaded = false;
   md->plan_key[0] = -1;
@@ -416,6 +462,12 @@ int sca_build_segment_mask_metadata_ex(sca_metadata* md, const sca_segment* cach
   md->pair_cost.swap(pair_cost);
   md->run_ptr.swap(run_ptr);
   md->runs.swap(runs);
+  md->kt_ptr.swap(kt_ptr);
+  md->kt_list.swap(kt_list);
+  md->kt_order.swap(kt_order);
+  md->qrun_ptr.swap(qrun_ptr);
+  md->qruns.swap(qruns);
+  md->kdesc_pad.swap(kdesc_pad);
   return SCA_OK;
 }
 
@@ -467,6 +519,13 @@ int sca_metadata_upload(sca_metadata* md, void* stream) {
   const size_t off_l = off;     off = align_up(off + std::max<size_t>(md->pair_list.size(), 1) * 4, 256);
   const size_t off_rp = off;    off = align_up(off + md->run_ptr.size() * 4, 256);
   const size_t off_r = off;     off = align_up(off + std::max<size_t>(md->runs.size(), 2) * 4, 256);
+  // backward lists (empty unless the layout has no cache)
+  const size_t off_ktp = off;   off = align_up(off + md->kt_ptr.size() * 4, 256);
+  const size_t off_ktl = off;   off = align_up(off + md->kt_list.size() * 4, 256);
+  const size_t off_kto = off;   off = align_up(off + md->kt_order.size() * 4, 256);
+  const size_t off_qrp = off;   off = align_up(off + md->qrun_ptr.size() * 4, 256);
+  const size_t off_qr = off;    off = align_up(off + md->qruns.size() * 4, 256);
+  const size_t off_kd = off;    off = align_up(off + md->kdesc_pad.size() * 4, 256);
   const size_t bytes = off;
 
   if (md->upload_done) {  // the staging buffer may still feed the previous copy
@@ -500,6 +559,12 @@ int sca_metadata_upload(sca_metadata* md, void* stream) {
   memcpy(h + off_l, md->pair_list.data(), md->pair_list.size() * 4);
   memcpy(h + off_rp, md->run_ptr.data(), md->run_ptr.size() * 4);
   memcpy(h + off_r, md->runs.data(), md->runs.size() * 4);
+  memcpy(h + off_ktp, md->kt_ptr.data(), md->kt_ptr.size() * 4);
+  memcpy(h + off_ktl, md->kt_list.data(), md->kt_list.size() * 4);
+  memcpy(h + off_kto, md->kt_order.data(), md->kt_order.size() * 4);
+  memcpy(h + off_qrp, md->qrun_ptr.data(), md->qrun_ptr.size() * 4);
+  memcpy(h + off_qr, md->qruns.data(), md->qruns.size() * 4);
+  memcpy(h + off_kd, md->kdesc_pad.data(), md->kdesc_pad.size() * 4);
   if (int rc = check_cuda(cudaMemcpyAsync(md->dev, h, bytes, cudaMemcpyHostToDevice, st),
                           "cudaMemcpyAsync(metadata)"))
     return rc;
@@ -510,6 +575,12 @@ int sca_metadata_upload(sca_metadata* md, void* stream) {
   md->off_list = off_l;
   md->off_run_ptr = off_rp;
   md->off_runs = off_r;
+  md->off_kt_ptr = off_ktp;
+  md->off_kt_list = off_ktl;
+  md->off_kt_order = off_kto;
+  md->off_qrun_ptr = off_qrp;
+  md->off_qruns = off_qr;
+  md->off_kdesc = off_kd;
   md->uploaded = true;
   return SCA_OK;
 }
@@ -916,6 +987,87 @@ int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md
   if (split)
     return check_cuda(launch_merge(a, static_cast<cudaStream_t>(stream)), "merge launch");
   return SCA_OK;
+}
+
+int sca_attn_bwd_workspace_bytes(const sca_metadata* md, int32_t heads, uint64_t* bytes) {
+  if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
+  if (heads < 1 || !bytes) return fail(SCA_ERR_INVALID_ARG, "need heads >= 1 and an output");
+  *bytes = 2ull * uint64_t(heads) * uint64_t(md->n_q_tiles) * SCA_TILE * 4;
+  return SCA_OK;
+}
+
+int sca_action_causal_attn_bwd(const sca_metadata* md, int32_t heads, const void* q, const void* k,
+                               const void* v, const void* o, const float* lse, const void* d_o,
+                               void* dq, void* dk, void* dv, float softmax_scale, void* workspace,
+                               uint64_t workspace_bytes, int32_t* dev_status, void* stream) {
+  if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
+  if (!md->uploaded) return fail(SCA_ERR_INVALID_ARG, "metadata not uploaded");
+  if (md->n_cached > 0)
+    return fail(SCA_ERR_UNSUPPORTED, "the backward pass takes layouts without cached segments");
+  if (heads < 1) return fail(SCA_ERR_INVALID_ARG, "heads must be >= 1");
+  if (!q || !k || !v || !o || !lse || !d_o || !dq || !dk || !dv)
+    return fail(SCA_ERR_INVALID_ARG, "null q, k, v, o, lse, d_o, dq, dk or dv");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(d_o) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(SCA_ERR_MISALIGNED, "tensors must be 16-byte aligned (lse 4-byte)");
+  if (!(softmax_scale > 0.f) || !isfinite(softmax_scale))
+    return fail(SCA_ERR_INVALID_ARG, "softmax_scale must be positive and finite");
+  uint64_t need = 0;
+  sca_attn_bwd_workspace_bytes(md, heads, &need);
+  if (!workspace || workspace_bytes < need)
+    return fail(SCA_ERR_CAPACITY, "the backward pass needs a workspace of %llu bytes",
+                (unsigned long long)need);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+    return fail(SCA_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+  int dev = 0;
+  if (int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice")) return rc;
+  if (dev != md->device) return fail(SCA_ERR_MISMATCH, "metadata was uploaded to another device");
+  if (int64_t(md->n_pairs) * 2 * heads > INT32_MAX) return fail(SCA_ERR_UNSUPPORTED, "grid too large");
+
+  const uint64_t n = uint64_t(md->n_q), n_pad = uint64_t(md->n_q_tiles) * SCA_TILE;
+  const uint64_t row = uint64_t(heads) * SCA_HEAD_DIM * 2;
+  BwdMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  int rc = make_map(&maps.q, q, uint64_t(heads), n, SCA_HEAD_DIM * 2, row, 1, SCA_TILE);
+  if (!rc) rc = make_map(&maps.k, k, uint64_t(heads), n, SCA_HEAD_DIM * 2, row, 1, SCA_TILE);
+  if (!rc) rc = make_map(&maps.v, v, uint64_t(heads), n, SCA_HEAD_DIM * 2, row, 1, SCA_TILE);
+  if (!rc) rc = make_map(&maps.d_o, d_o, uint64_t(heads), n, SCA_HEAD_DIM * 2, row, 1, SCA_TILE);
+  if (!rc) rc = make_scale_map(&maps.dl, static_cast<const float*>(workspace), n_pad,
+                               2 * uint64_t(heads), n_pad);
+  if (rc) return rc;
+
+  const uint8_t* d = static_cast<const uint8_t*>(md->dev);
+  BwdArgs a{};
+  a.item_order = reinterpret_cast<const int32_t*>(d + md->off_order);
+  a.pair_ptr = reinterpret_cast<const int32_t*>(d + md->off_ptr);
+  a.pair_list = reinterpret_cast<const uint32_t*>(d + md->off_list);
+  a.run_ptr = reinterpret_cast<const int32_t*>(d + md->off_run_ptr);
+  a.runs = reinterpret_cast<const uint2*>(d + md->off_runs);
+  a.qdesc = reinterpret_cast<const uint2*>(d + md->off_qdesc);
+  a.kt_order = reinterpret_cast<const int32_t*>(d + md->off_kt_order);
+  a.kt_ptr = reinterpret_cast<const int32_t*>(d + md->off_kt_ptr);
+  a.kt_list = reinterpret_cast<const uint32_t*>(d + md->off_kt_list);
+  a.qrun_ptr = reinterpret_cast<const int32_t*>(d + md->off_qrun_ptr);
+  a.qruns = reinterpret_cast<const uint4*>(d + md->off_qruns);
+  a.kdesc = reinterpret_cast<const uint32_t*>(d + md->off_kdesc);
+  a.o = o;
+  a.d_o = d_o;
+  a.lse = lse;
+  a.dl = static_cast<float*>(workspace);
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.status = dev_status;
+  a.n = int32_t(n);
+  a.n_pad = int32_t(n_pad);
+  a.heads = heads;
+  a.n_q_tiles = md->n_q_tiles;
+  a.n_pairs = md->n_pairs;
+  a.history = md->history;
+  a.scale = softmax_scale;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.timeout_ns = 2000000000ull;
+  return check_cuda(launch_backward(maps, a, static_cast<cudaStream_t>(stream)), "backward launch");
 }
 
 int sca_debug_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n, void* stream) {

@@ -120,6 +120,48 @@ struct AppendArgs {
 };
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
+
+// Attention backward (layouts without cached segments: keys = queries = the
+// n current tokens). Work-list views of the metadata, the workspace and the
+// tensors of one call.
+struct BwdArgs {
+  const int32_t* item_order;   // query-tile pairs, most expensive first
+  const int32_t* pair_ptr;     // [n_pairs + 1]
+  const uint32_t* pair_list;   // key tile | class of tile 0 << 24 | class of tile 1 << 26
+  const int32_t* run_ptr;      // key runs per key tile
+  const uint2* runs;
+  const uint2* qdesc;          // [n_pairs * 256] query descriptors
+  const int32_t* kt_order;     // key tiles, longest list first
+  const int32_t* kt_ptr;       // [n_kv_tiles + 1]
+  const uint32_t* kt_list;     // query tile | class << 24 (non-EMPTY only, ascending)
+  const int32_t* qrun_ptr;     // [n_q_tiles + 1] query runs per query tile
+  const uint4* qruns;          // {first | count << 8, query word 0, query word 1, 0}
+  const uint32_t* kdesc;       // [n_q_tiles * 128] key descriptor per token (0 past n)
+  const void* o;               // bf16 [n][heads][128]
+  const void* d_o;
+  const float* lse;            // [heads][n], natural log
+  float* dl;                   // workspace [2][heads][n_pad]: D, then LSE * log2(e)
+  void* dq;                    // bf16 [n][heads][128]
+  void* dk;
+  void* dv;
+  int32_t* status;
+  int32_t n;
+  int32_t n_pad;               // round_up(n, 128)
+  int32_t heads;
+  int32_t n_q_tiles;
+  int32_t n_pairs;
+  int32_t history;
+  float scale;
+  float scale_log2;
+  unsigned long long timeout_ns;
+};
+
+struct BwdMaps {
+  CUtensorMap q, k, v, d_o;    // token-major bf16, box (64, 1, 128)
+  CUtensorMap dl;              // workspace rows, box (128, 1)
+};
+
+cudaError_t launch_backward(const BwdMaps& maps, const BwdArgs& args, cudaStream_t stream);
 cudaError_t launch_bounded_wait(int32_t* status, unsigned long long timeout_ns,
                                 cudaStream_t stream);
 cudaError_t launch_exp2_eval(const float* x, float* y_poly, float* y_mufu, int64_t n,
@@ -156,6 +198,13 @@ struct sca_metadata {
   std::vector<float> pair_cost;        // [n_pairs] estimated cost (query-tile x key-tile units)
   std::vector<int32_t> run_ptr;        // [n_kv_tiles + 1]
   std::vector<uint32_t> runs;          // pairs of words: first | count << 8, descriptor
+  // backward (layouts without a cache only)
+  std::vector<int32_t> kt_ptr;         // [n_kv_tiles + 1]
+  std::vector<uint32_t> kt_list;       // query tile | class << 24
+  std::vector<int32_t> kt_order;       // key tiles, most expensive first
+  std::vector<int32_t> qrun_ptr;       // [n_q_tiles + 1]
+  std::vector<uint32_t> qruns;         // 4 words: first | count << 8, query words 0 and 1, 0
+  std::vector<uint32_t> kdesc_pad;     // [n_q_tiles * 128]
   // device copy
   bool uploaded = false;
   int device = -1;
@@ -166,6 +215,8 @@ struct sca_metadata {
   cudaEvent_t upload_done = nullptr;
   size_t off_qdesc = 0, off_order = 0, off_ptr = 0, off_list = 0;
   size_t off_run_ptr = 0, off_runs = 0;
+  size_t off_kt_ptr = 0, off_kt_list = 0, off_kt_order = 0, off_qrun_ptr = 0, off_qruns = 0,
+         off_kdesc = 0;
   // last split plan (heads, SMs, workspace, override) -> plan
   mutable int32_t plan_key[4] = {-1, -1, -1, -1};
   mutable uint64_t plan_ws = 0;

@@ -38,6 +38,7 @@ EXPORTED = (
     "sca_kv_cache_truncate", "sca_kv_cache_get", "sca_kv_cache_destroy",
     "sca_action_causal_attn_fwd", "sca_action_causal_attn_fwd_static_ws",
     "sca_attn_workspace_bytes", "sca_attn_plan",
+    "sca_action_causal_attn_bwd", "sca_attn_bwd_workspace_bytes",
     "sca_set_split_override",
     "sca_last_error", "sca_debug_bounded_wait", "sca_debug_exp2",
 )
@@ -90,6 +91,9 @@ _SIGS = {
     "sca_action_causal_attn_fwd_static_ws": [_P, _P, _i32, _P, _P, _P, _P, _P, ctypes.c_float,
                                              _P, _P],
     "sca_attn_workspace_bytes": [_P, _i32, ctypes.POINTER(ctypes.c_uint64)],
+    "sca_action_causal_attn_bwd": [_P, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_float,
+                                   _P, ctypes.c_uint64, _P, _P],
+    "sca_attn_bwd_workspace_bytes": [_P, _i32, ctypes.POINTER(ctypes.c_uint64)],
     "sca_attn_plan": [_P, _i32, _pi32, _pi32, _pi32],
     "sca_set_split_override": [_i32],
     "sca_last_error": [],
@@ -347,6 +351,29 @@ def action_causal_attn_fwd_static_ws(cache: Optional[KVCache], md: Metadata, hea
     _check(_lib.sca_action_causal_attn_fwd_static_ws(
         cache.handle if cache is not None else None, md.handle, int(heads), _ptr(q), _ptr(k_cur),
         _ptr(v_cur), _ptr(o), _ptr(lse), float(softmax_scale), _ptr(dev_status), _stream(stream)))
+
+
+def attn_bwd_workspace_bytes(md: Metadata, heads: int) -> int:
+    """Scratch bytes the backward needs (D and LSE·log2(e) per row)."""
+    b = ctypes.c_uint64()
+    _check(_lib.sca_attn_bwd_workspace_bytes(md.handle, int(heads), ctypes.byref(b)))
+    return int(b.value)
+
+
+def action_causal_attn_bwd(md: Metadata, heads: int, q, k, v, o, lse, d_o, dq, dk, dv,
+                           softmax_scale: float = 128 ** -0.5, workspace=None,
+                           workspace_bytes: Optional[int] = None, dev_status=None,
+                           stream=None) -> None:
+    """Gradients dq, dk, dv (written) of the forward for upstream gradient
+    d_o; ``workspace``: a uint8 device tensor (or an int address with
+    ``workspace_bytes``) of at least ``attn_bwd_workspace_bytes``."""
+    if workspace is not None and workspace_bytes is None:
+        workspace_bytes = int(workspace.numel() * workspace.element_size())
+    _check(_lib.sca_action_causal_attn_bwd(md.handle, int(heads), _ptr(q), _ptr(k), _ptr(v),
+                                           _ptr(o), _ptr(lse), _ptr(d_o), _ptr(dq), _ptr(dk),
+                                           _ptr(dv), float(softmax_scale), _ptr(workspace),
+                                           int(workspace_bytes or 0), _ptr(dev_status),
+                                           _stream(stream)))
 
 
 def attn_workspace_bytes(md: Metadata, heads: int) -> int:
