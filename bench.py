@@ -52,6 +52,11 @@ WORKLOADS = {
                                                           name="480p-long-session-int8"),
 }
 INT8_WORKLOADS = {"480p-long-session-int8"}
+# the backward of the packed training batch (the forward that produces O and
+# LSE runs once, untimed; a step is one backward call)
+WORKLOADS["packed-360k-bwd"] = lambda: dataclasses.replace(W.packed_360k(), name="packed-360k-bwd")
+BWD_WORKLOADS = {"packed-360k-bwd"}
+BWD_FLOP_FACTOR = 2.5   # five products per visible pair against the forward's two
 KERNEL_SOURCES = ["segment_causal_masked_b200/csrc/sca_kernels.cu",
                   "segment_causal_masked_b200/csrc/sca_internal.h"]
 
@@ -155,7 +160,8 @@ class OracleSample:
     """The oracle on `rows` query rows (spread evenly over the query tiles) and
     `heads` head(s) of the workload, inputs drawn once."""
 
-    def __init__(self, problem, rows: int, heads: int = 1, seed: int = 7, int8: bool = False):
+    def __init__(self, problem, rows: int, heads: int = 1, seed: int = 7, int8: bool = False,
+                 backward: bool = False):
         import numpy as np
         import torch
 
@@ -175,16 +181,25 @@ class OracleSample:
             self.k[:nc] = ocache.dequantize_rows(*ocache.quantize_rows(self.k[:nc]))
             self.v[:nc] = ocache.dequantize_rows(*ocache.quantize_rows(self.v[:nc]))
         self.pairs = sum(sum(b - a for a, b in self.lay.ranges(int(r))) for r in self.rows)
-        self.flops = 4.0 * W.HEAD_DIM * heads * self.pairs
+        self.backward = backward
+        self.flops = (6.0 if backward else 4.0) * W.HEAD_DIM * heads * self.pairs
         self.desc = (f"oracle (float64 NumPy) on {rows} query rows x {heads} head(s) of "
                      f"{problem.name} ({self.pairs} unmasked pairs per head), as effective "
-                     f"TFLOP/s of that sample")
+                     f"TFLOP/s of that sample"
+                     + (": the dQ rows (three products per visible pair: S, dP, dS K)"
+                        if backward else ""))
+        if backward:
+            self.d_o = W.randn_bf16((nq, heads, W.HEAD_DIM), 1000 * seed + 3).float().numpy()
 
     def run(self) -> float:
         from oracle import attention as oattn
+        from oracle import backward as obwd
 
         t0 = time.perf_counter()
-        oattn.attention_rows(self.lay, self.q, self.k, self.v, self.rows, self.p.softmax_scale)
+        if self.backward:
+            obwd.dq_rows(self.lay, self.q, self.k, self.v, self.d_o, self.rows, self.p.softmax_scale)
+        else:
+            oattn.attention_rows(self.lay, self.q, self.k, self.v, self.rows, self.p.softmax_scale)
         return time.perf_counter() - t0
 
 
@@ -204,13 +219,15 @@ def run_reference(args, problem):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    sample = OracleSample(problem, args.oracle_rows, int8=args.workload in INT8_WORKLOADS)
+    bwd = args.workload in BWD_WORKLOADS
+    sample = OracleSample(problem, args.oracle_rows // (8 if bwd else 1),
+                          int8=args.workload in INT8_WORKLOADS, backward=bwd)
     for _ in range(args.warmup):
         sample.run()
     secs = [sample.run() for _ in range(args.steps)]
     vals = [sample.flops / s / 1e12 for s in secs]
     desc = sample.desc
-    rows_per_step = args.oracle_rows
+    rows_per_step = len(sample.rows)
     value = statistics.mean(vals)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -301,6 +318,39 @@ class Session:
         self.stream = torch.cuda.current_stream()
         torch.cuda.synchronize()
 
+    def prepare_backward(self, seed: int):
+        """One forward (O, LSE), an upstream gradient dO, gradient outputs and
+        the backward's workspace."""
+        import torch
+
+        sca, p = self.sca, self.p
+        dev = self.q.device
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed)
+        self.md.upload(self.stream.cuda_stream)
+        sca.action_causal_attn_fwd(None, self.md, p.heads, self.q, self.k_cur, self.v_cur, self.o,
+                                   self.lse, p.softmax_scale, self.workspace, None, self.status,
+                                   self.stream.cuda_stream)
+        self.d_o = torch.randn(self.q.shape, generator=g, device=dev).to(torch.bfloat16)
+        self.dq, self.dk, self.dv = (torch.empty_like(self.q) for _ in range(3))
+        self.bws = torch.empty(sca.attn_bwd_workspace_bytes(self.md, p.heads), dtype=torch.uint8,
+                               device=dev)
+        torch.cuda.synchronize()
+
+    def step_backward(self, q=None, k=None, v=None, o=None, lse=None, d_o=None, ev=None):
+        """One backward call; `ev` = (start, end) events around it."""
+        sca, p = self.sca, self.p
+        s = self.stream.cuda_stream
+        if ev is not None:
+            ev[0].record(self.stream)
+        sca.action_causal_attn_bwd(self.md, p.heads, self.q if q is None else q,
+                                   self.k_cur if k is None else k, self.v_cur if v is None else v,
+                                   self.o if o is None else o, self.lse if lse is None else lse,
+                                   self.d_o if d_o is None else d_o, self.dq, self.dk, self.dv,
+                                   p.softmax_scale, self.bws, None, self.status, s)
+        if ev is not None:
+            ev[1].record(self.stream)
+
     def step(self, q=None, k_cur=None, v_cur=None, o=None, ev=None):
         """One pass of the hot path; `ev` = (start, end) events around the
         attention kernel."""
@@ -346,16 +396,22 @@ def run_native(args, problem):
         return reduce_max(x, world, "cuda")
 
     int8 = args.workload in INT8_WORKLOADS
+    bwd = args.workload in BWD_WORKLOADS
     sess = Session(problem, seed=1000 * 2 + rank, int8=int8)
     from segment_causal_masked_b200 import sca
     sca_md = sca.build_for(problem)
     counts = sca_md.counts()
     A = counts["unmasked_pairs"]
     flops = effective_flops(problem, A)
+    step = sess.step
+    if bwd:
+        sess.prepare_backward(1000 * 3 + rank)
+        flops *= BWD_FLOP_FACTOR
+        step = sess.step_backward
 
     # ---- device-resident timing
     for _ in range(args.warmup):
-        sess.step()
+        step()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
@@ -366,7 +422,7 @@ def run_native(args, problem):
     clocks.start()
     t_start.record(sess.stream)
     for i in range(args.steps):
-        sess.step(ev=evs[i])
+        step(ev=evs[i])
     t_end.record(sess.stream)
     torch.cuda.synchronize()
     clock_info = clocks.stop()
@@ -395,6 +451,23 @@ def run_native(args, problem):
         sess.step(q=dq, k_cur=dk, v_cur=dv)
         ho.copy_(sess.o, non_blocking=True)
 
+    bytes_in = 3 * hq.numel() * hq.element_size()
+    bytes_out = ho.numel() * ho.element_size()
+    if bwd:  # inputs q, k, v, o, lse, dO in; dq, dk, dv out
+        h_o, h_do, h_lse = sess.o.cpu().pin_memory(), sess.d_o.cpu().pin_memory(), sess.lse.cpu().pin_memory()
+        d_o_, d_do, d_lse = torch.empty_like(sess.o), torch.empty_like(sess.d_o), torch.empty_like(sess.lse)
+        h_g = [torch.empty(nq, h, 128, **pin) for _ in range(3)]
+
+        def e2e_step():  # noqa: F811
+            for dst, src in ((dq, hq), (dk, hk), (dv, hv), (d_o_, h_o), (d_do, h_do), (d_lse, h_lse)):
+                dst.copy_(src, non_blocking=True)
+            sess.step_backward(q=dq, k=dk, v=dv, o=d_o_, lse=d_lse, d_o=d_do)
+            for dst, src in zip(h_g, (sess.dq, sess.dk, sess.dv)):
+                dst.copy_(src, non_blocking=True)
+
+        bytes_in = 5 * hq.numel() * hq.element_size() + h_lse.numel() * 4
+        bytes_out = 3 * hq.numel() * hq.element_size()
+
     for _ in range(args.warmup):
         e2e_step()
     torch.cuda.synchronize()
@@ -408,14 +481,12 @@ def run_native(args, problem):
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
     e2e_value = whole_job_tflops(world, flops, args.steps, e2e_ms)
-    bytes_in = 3 * hq.numel() * hq.element_size()
-    bytes_out = ho.numel() * ho.element_size()
 
     if rank == 0:
         peaks = measured_peaks()
         peak = float(peaks["bf16_tflops"])
         achieved = flops / (attn_avg * 1e-3) / 1e12
-        traffic = stored_traffic("attn_fwd_kernel", problem.name)
+        traffic = None if bwd else stored_traffic("attn_fwd_kernel", problem.name)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -425,8 +496,12 @@ def run_native(args, problem):
                        "cached_segments": len(problem.cached), "heads": h,
                        "head_dim": W.HEAD_DIM, "unmasked_pairs_per_head": A,
                        "effective_flop_per_step": flops,
-                       "step": ("metadata build+upload, attention forward, kv_cache_append"
+                       "step": ("attention backward (D and LSE, dQ, dK and dV kernels); the "
+                                "forward that produced O and LSE ran once before timing" if bwd
+                                else "metadata build+upload, attention forward, kv_cache_append"
                                 if sess.appends else "metadata build+upload, attention forward"),
+                       "flop_count": ("10·d·H·A (five products per visible pair)" if bwd
+                                      else "4·d·H·A (two products per visible pair)"),
                        "kv_cache": "int8 codes + fp32 row scales" if int8 else "bf16",
                        "l2": "inputs larger than L2 (cached K/V %.2f GB per tensor)"
                              % (problem.n_cache_tokens * h * (132 if int8 else 256) / 1e9),
@@ -435,15 +510,17 @@ def run_native(args, problem):
             "pct_of_peak": 100.0 * value / world / peak,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "attn_fwd_kernel", "kernel_ms": attn_avg,
+                         "kernel": ("bwd_prep_kernel + bwd_dq_kernel + bwd_dkdv_kernel" if bwd
+                                    else "attn_fwd_kernel"), "kernel_ms": attn_avg,
                          "peak_source": f"{peaks['source']} bf16 dense (burst)"},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": bytes_in,
                     "d2h_bytes_per_step": bytes_out, "ms_per_step": e2e_ms / args.steps},
-            "gpu_launches": (1 + int(sess.appends) + int(sess.splits)) * args.steps,
+            "gpu_launches": (3 if bwd else 1 + int(sess.appends) + int(sess.splits)) * args.steps,
             "clocks": clock_info,
         }
         if not args.no_cpu_baseline:
-            sample = OracleSample(problem, args.baseline_rows, int8=int8)
+            sample = OracleSample(problem, args.baseline_rows // (8 if bwd else 1), int8=int8,
+                                  backward=bwd)
             dt = sample.run()
             line["cpu_baseline"] = {"value": sample.flops / dt / 1e12, "unit": "TFLOP/s",
                                     "cores": cpu_threads(), "kind": "oracle",
