@@ -338,7 +338,7 @@ SCA_API int sca_action_causal_attn_fwd_static_ws(const sca_kv_cache* cache,
  *   dq, dk, dv : bf16 [n][heads][128], written (not accumulated);
  *   workspace, workspace_bytes : device scratch of at least
  *            sca_attn_bwd_workspace_bytes (256-byte aligned; required:
- *            SCA_ERR_CAPACITY otherwise); it receives D and LSE·log2(e);
+ *            SCA_ERR_CAPACITY otherwise); it receives −D and −LSE·log2(e);
  *   dev_status, stream : as for the forward.
  * Three kernels on the stream: D and LSE, dQ (query tiles over their key
  * tiles), dK and dV (key tiles over the query tiles that see them); no

@@ -84,21 +84,28 @@ __device__ __forceinline__ void set_run_bits(uint32_t (&vis)[2], int a, int b, i
   }
 }
 
-// p = exp2(s * scale_log2 - l) where visible (0 elsewhere), ds = p (dp - d);
-// 64 columns -> 32 bf16 pairs of p and of ds.
-__device__ __forceinline__ void p_ds_row(const float (&s)[64], const float (&dp)[64],
-                                         const uint32_t (&vis)[2], bool full, float scale_log2,
-                                         float l, float d, uint32_t (&pw)[32], uint32_t (&dsw)[32]) {
+// ds = p (dp - d) with p = exp2(s * scale_log2 - l) where visible (0
+// elsewhere), for 32 columns given as pairs; nl2 = (-l, -l), nd2 = (-d, -d)
+// per column pair. Packed fp32 pairs; bf16 pairs of ds out.
+template <bool kFull>
+__device__ __forceinline__ void ds_pairs(const float (&s)[32], const float (&dp)[32],
+                                         uint32_t vis, uint64_t c2, const uint64_t* nl2,
+                                         const uint64_t* nd2, uint32_t (&dsw)[16],
+                                         uint32_t* pw = nullptr) {
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    float p0 = ex2(fmaf(s[2 * i], scale_log2, -l));
-    float p1 = ex2(fmaf(s[2 * i + 1], scale_log2, -l));
-    if (!full) {
-      p0 = ((vis[(2 * i) >> 5] >> ((2 * i) & 31)) & 1u) ? p0 : 0.f;
-      p1 = ((vis[(2 * i + 1) >> 5] >> ((2 * i + 1) & 31)) & 1u) ? p1 : 0.f;
+  for (int i = 0; i < 16; ++i) {
+    float x0, x1;
+    unf2(fma2(f2(s[2 * i], s[2 * i + 1]), c2, nl2[i]), x0, x1);
+    float p0 = ex2(x0), p1 = ex2(x1);
+    if (!kFull) {
+      p0 = ((vis >> (2 * i)) & 1u) ? p0 : 0.f;
+      p1 = ((vis >> (2 * i + 1)) & 1u) ? p1 : 0.f;
     }
-    pw[i] = pack_bf16(p0, p1);
-    dsw[i] = pack_bf16(p0 * (dp[2 * i] - d), p1 * (dp[2 * i + 1] - d));
+    const uint64_t pp = f2(p0, p1);
+    float d0, d1;
+    unf2(mul2(pp, add2(f2(dp[2 * i], dp[2 * i + 1]), nd2[i])), d0, d1);
+    dsw[i] = pack_bf16(d0, d1);
+    if (pw) pw[i] = pack_bf16(p0, p1);
   }
 }
 
@@ -108,10 +115,10 @@ __device__ __forceinline__ void p_ds_row(const float (&s)[64], const float (&dp)
 // D = rowsum(dO ∘ O) and LSE · log2(e), per (head, query)
 // ---------------------------------------------------------------------------
 
-// One warp per (query, head) row, 4 values per lane. Rows past n (up to the
-// tile-padded n_pad) get D = 0 and L = 0; the kernels never use them
-// unmasked. A row with LSE = -inf (it sees nothing) gets L = +inf, so that
-// its probabilities come out 0.
+// One warp per (query, head) row, 4 values per lane; the workspace receives
+// -D and -L (L = LSE · log2 e). Rows past n (up to the tile-padded n_pad) get
+// 0; the kernels never use them unmasked. A row with LSE = -inf (it sees
+// nothing) gets L = +inf, so that its probabilities come out 0.
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
   const uint2* __restrict__ o = static_cast<const uint2*>(a.o);
   const uint2* __restrict__ g = static_cast<const uint2*>(a.d_o);
@@ -135,9 +142,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdArgs a) {
       const float lse = a.lse[int64_t(h) * a.n + tok];
       l = lse == -INFINITY ? INFINITY : lse * kLog2e;
     }
-    if (lane == 0) {
-      a.dl[int64_t(h) * a.n_pad + tok] = d;
-      a.dl[int64_t(a.heads + h) * a.n_pad + tok] = l;
+    if (lane == 0) {  // stored negated: the kernels add them with packed FMAs
+      a.dl[int64_t(h) * a.n_pad + tok] = -d;
+      a.dl[int64_t(a.heads + h) * a.n_pad + tok] = -l;
     }
   }
 }
@@ -334,8 +341,15 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const int q_row = qtile * 128 + r;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const uint2 qd = p.qdesc[q_row];
-    const float l = p.dl[int64_t(p.heads + head) * p.n_pad + q_row];
-    const float d = p.dl[int64_t(head) * p.n_pad + q_row];
+    const float nl = p.dl[int64_t(p.heads + head) * p.n_pad + q_row];  // -L
+    const float nd = p.dl[int64_t(head) * p.n_pad + q_row];            // -D
+    uint64_t nl2[16], nd2[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      nl2[i] = f2(nl, nl);
+      nd2[i] = f2(nd, nd);
+    }
+    const uint64_t c2 = f2(p.scale_log2, p.scale_log2);
     const int c0 = 64 * half;
     bool ok = true;
     int j = 0;
@@ -366,8 +380,15 @@ __global__ void __launch_bounds__(kBThreads, 1)
       tmem_ld32(tDP + lane_base + c0, dp);
       tmem_ld32(tDP + lane_base + c0 + 32, dp + 32);
       tmem_wait_ld();
-      uint32_t pw[32], dsw[32];
-      p_ds_row(s, dp, vis, cls == SCA_TILE_FULL, p.scale_log2, l, d, pw, dsw);
+      uint32_t dsw[32];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float(&sh)[32] = *reinterpret_cast<const float(*)[32]>(s + 32 * h);
+        const float(&dph)[32] = *reinterpret_cast<const float(*)[32]>(dp + 32 * h);
+        uint32_t(&out)[16] = *reinterpret_cast<uint32_t(*)[16]>(dsw + 16 * h);
+        if (cls == SCA_TILE_FULL) ds_pairs<true>(sh, dph, 0u, c2, nl2, nd2, out);
+        else ds_pairs<false>(sh, dph, vis[h], c2, nl2, nd2, out);
+      }
       tmem_st16(tSj + c0, dsw);  // dS over the first 32 columns of this half
       tmem_st16(tSj + c0 + 16, dsw + 16);
       tmem_wait_st();
@@ -554,6 +575,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const uint32_t kd = p.kdesc[key];
     const int c0 = 64 * half;
+    const uint64_t c2 = f2(p.scale_log2, p.scale_log2);
     bool ok = true;
     int i = 0;
     for (; i < n; ++i) {
@@ -577,31 +599,27 @@ __global__ void __launch_bounds__(kBThreads, 1)
         break;
       }
       tc_fence_after();
-      float s[64], dp[64];
-      tmem_ld32(tSt + lane_base + c0, s);
-      tmem_ld32(tSt + lane_base + c0 + 32, s + 32);
-      tmem_ld32(tDPt + lane_base + c0, dp);
-      tmem_ld32(tDPt + lane_base + c0 + 32, dp + 32);
-      const float* dl = reinterpret_cast<const float*>(smem + stage(i) + 2 * kBTile);
-      tmem_wait_ld();
+      // per column (query) -D and -L, as pairs, half by half: 32 columns of
+      // S, dP and of the two vectors are live at a time
+      const uint64_t* ndl = reinterpret_cast<const uint64_t*>(smem + stage(i) + 2 * kBTile);
       uint32_t pw[32], dsw[32];
 #pragma unroll
-      for (int c = 0; c < 64; c += 4) {  // per column: this query's D and L
-        const float4 dd = *reinterpret_cast<const float4*>(dl + c0 + c);
-        const float4 ll = *reinterpret_cast<const float4*>(dl + 128 + c0 + c);
-        const float dv4[4] = {dd.x, dd.y, dd.z, dd.w}, lv4[4] = {ll.x, ll.y, ll.z, ll.w};
+      for (int h = 0; h < 2; ++h) {
+        const int cb = c0 + 32 * h;
+        float s[32], dp[32];
+        tmem_ld32(tSt + lane_base + cb, s);
+        tmem_ld32(tDPt + lane_base + cb, dp);
+        uint64_t nd2[16], nl2[16];
 #pragma unroll
-        for (int u = 0; u < 4; u += 2) {
-          const int cc = c + u;
-          float p0 = ex2(fmaf(s[cc], p.scale_log2, -lv4[u]));
-          float p1 = ex2(fmaf(s[cc + 1], p.scale_log2, -lv4[u + 1]));
-          if (cls != SCA_TILE_FULL) {
-            p0 = ((vis[cc >> 5] >> (cc & 31)) & 1u) ? p0 : 0.f;
-            p1 = ((vis[(cc + 1) >> 5] >> ((cc + 1) & 31)) & 1u) ? p1 : 0.f;
-          }
-          pw[cc >> 1] = pack_bf16(p0, p1);
-          dsw[cc >> 1] = pack_bf16(p0 * (dp[cc] - dv4[u]), p1 * (dp[cc + 1] - dv4[u + 1]));
+        for (int k = 0; k < 16; ++k) {
+          nd2[k] = ndl[cb / 2 + k];
+          nl2[k] = ndl[64 + cb / 2 + k];
         }
+        tmem_wait_ld();
+        uint32_t(&po)[16] = *reinterpret_cast<uint32_t(*)[16]>(pw + 16 * h);
+        uint32_t(&dso)[16] = *reinterpret_cast<uint32_t(*)[16]>(dsw + 16 * h);
+        if (cls == SCA_TILE_FULL) ds_pairs<true>(s, dp, 0u, c2, nl2, nd2, dso, po);
+        else ds_pairs<false>(s, dp, vis[h], c2, nl2, nd2, dso, po);
       }
       tmem_st16(tSt + lane_base + c0, pw);  // Pᵀ over the first 32 columns of this half
       tmem_st16(tSt + lane_base + c0 + 16, pw + 16);
