@@ -74,6 +74,42 @@ __device__ __forceinline__ void mma_ts8_split(uint32_t d_tmem, uint32_t a_lo, ui
       : "memory");
 }
 
+// D (+)= A B with A from TMEM laid out by the dK/dV kernel: the 16-query
+// K-step k sits at column a + {0, 8, 32, 40, 16, 24, 48, 56}[k] (warpgroup
+// (k/2) % 2 wrote queries [64 b, 64 b + 64) of its 32-column blocks at
+// 32 w + 16 b); B MN-major, 2048 B per K-step.
+__device__ __forceinline__ void mma_ts8_blocks(uint32_t d_tmem, uint32_t a, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred pf, pt;\n\t.reg .b32 ta, bl;\n\t.reg .b64 bd;\n\t"
+      "setp.ne.b32 pf, %5, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\t"
+      "mov.b64 bd, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, pf;\n\t"
+      "add.u32 ta, %1, 8;\n\tadd.u32 bl, %2, 128;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %4, pt;\n\t"
+      "add.u32 ta, %1, 32;\n\tadd.u32 bl, %2, 256;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %4, pt;\n\t"
+      "add.u32 ta, %1, 40;\n\tadd.u32 bl, %2, 384;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %4, pt;\n\t"
+      "add.u32 ta, %1, 16;\n\tadd.u32 bl, %2, 512;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %4, pt;\n\t"
+      "add.u32 ta, %1, 24;\n\tadd.u32 bl, %2, 640;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %4, pt;\n\t"
+      "add.u32 ta, %1, 48;\n\tadd.u32 bl, %2, 768;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %4, pt;\n\t"
+      "add.u32 ta, %1, 56;\n\tadd.u32 bl, %2, 896;\n\tmov.b64 bd, {bl, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], bd, %4, pt;\n\t}"
+      ::"r"(d_tmem), "r"(a), "r"(uint32_t(b_desc)), "r"(uint32_t(b_desc >> 32)), "r"(idesc),
+      "r"(acc)
+      : "memory");
+}
+
+// Columns [c0, c0 + 32) of a run [a, b) as a 32-bit mask.
+__device__ __forceinline__ uint32_t run_bits32(int a, int b, int c0) {
+  const int lo = max(a, c0) - c0, hi = min(b, c0 + 32) - c0;
+  return lo < hi ? uint32_t(((1ull << (hi - lo)) - 1ull) << lo) : 0u;
+}
+
 // Columns [c0, c0 + 64) of a run [a, b) as two 32-bit masks.
 __device__ __forceinline__ void set_run_bits(uint32_t (&vis)[2], int a, int b, int c0) {
 #pragma unroll
@@ -160,7 +196,8 @@ constexpr int kQKSlots = 3, kQVSlots = 2;
 constexpr uint32_t kQBarQD = 0, kQBarKF = 1, kQBarKE = kQBarKF + kQKSlots,
                    kQBarVF = kQBarKE + kQKSlots, kQBarVE = kQBarVF + kQVSlots,
                    kQBarS = kQBarVE + kQVSlots, kQBarDP = kQBarS + 2, kQBarDS = kQBarDP + 1,
-                   kQBarDone = kQBarDS + 1, kQBarDrain = kQBarDone + 1, kQNumBars = kQBarDrain + 1;
+                   kQBarRD = kQBarDS + 1, kQBarDone = kQBarRD + 1, kQBarDrain = kQBarDone + 1,
+                   kQNumBars = kQBarDrain + 1;
 constexpr uint32_t kQOffBar = 7 * kBTile;
 constexpr uint32_t kQOffCtl = kQOffBar + kQNumBars * 8;
 constexpr uint32_t kQOffSlot = kQOffCtl + 16;
@@ -205,6 +242,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     mbar_init(bar(kQBarS + 1), 1);
     mbar_init(bar(kQBarDP), 1);
     mbar_init(bar(kQBarDS), 256);
+    mbar_init(bar(kQBarRD), 256);
     mbar_init(bar(kQBarDone), 1);
     mbar_init(bar(kQBarDrain), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -309,15 +347,19 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
         for (int j = 0; ok && j < n; ++j) {
           const uint32_t tSj = tS0 + uint32_t(j & 1) * 128;
-          if (!(ok = wait_bar(bar(kQBarDS), uint32_t(j) & 1u, ctl, p.status, p.timeout_ns))) break;
+          // dP of the next key tile as soon as dP_j has been read out: it
+          // overlaps the elementwise work on this one
+          if (!(ok = wait_bar(bar(kQBarRD), uint32_t(j) & 1u, ctl, p.status, p.timeout_ns))) break;
           tc_fence_after();
-          if (j + 1 < n) {  // dP of the next key tile first: the elementwise warps wait on it
+          if (j + 1 < n) {
             if (!(ok = wait_v(j + 1))) break;
             tc_fence_after();
             mma_qk8(tDP, dDO, desc_kmajor(vslot(j + 1)), kIdescQK);
             mma_commit(bar(kQBarDP));
             mma_commit(bar(kQBarVE + (j + 1) % kQVSlots));
           }
+          if (!(ok = wait_bar(bar(kQBarDS), uint32_t(j) & 1u, ctl, p.status, p.timeout_ns))) break;
+          tc_fence_after();
           mma_ts8_split(tDQ, tSj, tSj + 64, desc_mnmajor(kslot(j)), kIdescPV, j > 0 ? 1u : 0u);
           mma_commit(bar(kQBarKE + j % kQKSlots));
           if (j + 2 < n) {  // S of the key tile after next into the slot dS_j leaves
@@ -380,6 +422,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
       tmem_ld32(tDP + lane_base + c0, dp);
       tmem_ld32(tDP + lane_base + c0 + 32, dp + 32);
       tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(kQBarRD));  // dP_j is in registers: the next dP may overwrite it
       uint32_t dsw[32];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -438,9 +482,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
 constexpr uint32_t kKOffK = 0, kKOffV = kBTile, kKOffStage = 2 * kBTile;
 constexpr uint32_t kKStage = 2 * kBTile + 1024;  // Q, dO, D[128], L[128]
 constexpr int kKStages = 2;
-constexpr uint32_t kKBarKV = 0, kKBarF = 1, kKBarE = kKBarF + kKStages, kKBarSDP = kKBarE + kKStages,
-                   kKBarDS = kKBarSDP + 1, kKBarDone = kKBarDS + 1, kKBarDrain = kKBarDone + 1,
-                   kKNumBars = kKBarDrain + 1;
+constexpr uint32_t kKBarKV = 0, kKBarF = 1, kKBarE = kKBarF + kKStages, kKBarST = kKBarE + kKStages,
+                   kKBarDPT = kKBarST + 1, kKBarRD = kKBarDPT + 1, kKBarDS = kKBarRD + 1,
+                   kKBarDone = kKBarDS + 1, kKBarDrain = kKBarDone + 1, kKNumBars = kKBarDrain + 1;
 constexpr uint32_t kKOffBar = kKOffStage + kKStages * kKStage;
 constexpr uint32_t kKOffCtl = kKOffBar + kKNumBars * 8;
 constexpr uint32_t kKOffSlot = kKOffCtl + 16;
@@ -476,7 +520,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
       mbar_init(bar(kKBarF + s), 1);
       mbar_init(bar(kKBarE + s), 1);
     }
-    mbar_init(bar(kKBarSDP), 1);
+    mbar_init(bar(kKBarST), 1);
+    mbar_init(bar(kKBarDPT), 1);
+    mbar_init(bar(kKBarRD), 256);
     mbar_init(bar(kKBarDS), 256);
     mbar_init(bar(kKBarDone), 1);
     mbar_init(bar(kKBarDrain), 1);
@@ -535,31 +581,39 @@ __global__ void __launch_bounds__(kBThreads, 1)
         return wait_bar(bar(kKBarF + i % kKStages), uint32_t(i / kKStages) & 1u, ctl, p.status,
                         p.timeout_ns);
       };
-      auto issue_sdp = [&](int i) {  // Sᵀ = K Qᵢᵀ, dPᵀ = V dOᵢᵀ
-        const uint32_t st = sbase + stage(i);
-        mma_qk8(tSt, dK, desc_kmajor(st), kIdescQK);
-        mma_qk8(tDPt, dV, desc_kmajor(st + kBTile), kIdescQK);
-        mma_commit(bar(kKBarSDP));
+      auto issue_s = [&](int i) {  // Sᵀ = K Qᵢᵀ
+        mma_qk8(tSt, dK, desc_kmajor(sbase + stage(i)), kIdescQK);
+        mma_commit(bar(kKBarST));
+      };
+      auto issue_dp = [&](int i) {  // dPᵀ = V dOᵢᵀ
+        mma_qk8(tDPt, dV, desc_kmajor(sbase + stage(i) + kBTile), kIdescQK);
+        mma_commit(bar(kKBarDPT));
       };
       // K and V are always loaded: wait for them even with no query tile
       bool ok = wait_bar(bar(kKBarKV), 0, ctl, p.status, p.timeout_ns) && (n == 0 || wait_f(0));
       if (ok && n > 0) {
         tc_fence_after();
-        issue_sdp(0);
+        issue_s(0);
+        issue_dp(0);
       }
       for (int i = 0; ok && i < n; ++i) {
+        // the next dPᵀ as soon as this one has been read out (the elementwise
+        // warps write Pᵀ and dSᵀ into the Sᵀ columns only)
+        if (!(ok = wait_bar(bar(kKBarRD), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns))) break;
+        tc_fence_after();
+        if (i + 1 < n) {
+          if (!(ok = wait_f(i + 1))) break;
+          tc_fence_after();
+          issue_dp(i + 1);
+        }
         if (!(ok = wait_bar(bar(kKBarDS), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns))) break;
         tc_fence_after();
         const uint32_t st = sbase + stage(i);
         // dV += Pᵀ dO, dK += dSᵀ Q (B MN-major: rows are queries)
-        mma_ts8_split(tDV, tSt, tSt + 64, desc_mnmajor(st + kBTile), kIdescPV, i > 0 ? 1u : 0u);
-        mma_ts8_split(tDK, tDPt, tDPt + 64, desc_mnmajor(st), kIdescPV, i > 0 ? 1u : 0u);
+        mma_ts8_blocks(tDV, tSt, desc_mnmajor(st + kBTile), kIdescPV, i > 0 ? 1u : 0u);
+        mma_ts8_blocks(tDK, tSt + 64, desc_mnmajor(st), kIdescPV, i > 0 ? 1u : 0u);
         mma_commit(bar(kKBarE + i % kKStages));
-        if (i + 1 < n) {
-          if (!(ok = wait_f(i + 1))) break;
-          tc_fence_after();
-          issue_sdp(i + 1);
-        }
+        if (i + 1 < n) issue_s(i + 1);
       }
       mma_commit(bar(kKBarDone));
       mma_commit(bar(kKBarDrain));
@@ -569,12 +623,12 @@ __global__ void __launch_bounds__(kBThreads, 1)
   } else {
     // ------------------------------------------------------------------ elementwise
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kBRegsWork));
-    const int half = warp >> 2;                   // query columns [64 half, 64 half + 64)
+    const int half = warp >> 2;                   // query blocks [32 half, +32), [64 + 32 half, +32)
     const int r = (warp & 3) * 32 + lane;         // key row = TMEM lane
     const int key = ktile * 128 + r;
     const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
     const uint32_t kd = p.kdesc[key];
-    const int c0 = 64 * half;
+    const int c0 = 64 * half;                     // output columns of this half (epilogue)
     const uint64_t c2 = f2(p.scale_log2, p.scale_log2);
     bool ok = true;
     int i = 0;
@@ -582,49 +636,60 @@ __global__ void __launch_bounds__(kBThreads, 1)
       const uint32_t e = list[i];
       const int qt = int(e & kPairTileMask);
       const uint32_t cls = e >> 24;
-      uint32_t vis[2] = {0u, 0u};
+      uint32_t vis[2] = {0u, 0u};  // query blocks b = 0, 1
       if (cls == SCA_TILE_PARTIAL && key < p.n) {  // a padding key sees nothing
         for (int k = p.qrun_ptr[qt]; k < p.qrun_ptr[qt + 1]; ++k) {
           const uint4 run = p.qruns[k];
           if (!visible(run.y, run.z, kd, uint32_t(p.history))) continue;
-          const int a = int(run.x & 255u);
-          set_run_bits(vis, a, a + int((run.x >> 8) & 255u), c0);
+          const int a = int(run.x & 255u), b = a + int((run.x >> 8) & 255u);
+          vis[0] |= run_bits32(a, b, 32 * half);
+          vis[1] |= run_bits32(a, b, 64 + 32 * half);
         }
       }
       ok = wait_bar(bar(kKBarF + i % kKStages), uint32_t(i / kKStages) & 1u, ctl, p.status,
                     p.timeout_ns) &&
-           wait_bar(bar(kKBarSDP), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns);
+           wait_bar(bar(kKBarDPT), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns);
       if (!__all_sync(0xFFFFFFFFu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // per column (query) -D and -L, as pairs, half by half: 32 columns of
-      // S, dP and of the two vectors are live at a time
+      float dp[64], s[64];
+      tmem_ld32(tDPt + lane_base + 32 * half, dp);
+      tmem_ld32(tDPt + lane_base + 64 + 32 * half, dp + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(kKBarRD));  // dPᵀ is in registers: the next dPᵀ may overwrite it
+      if (!__all_sync(0xFFFFFFFFu, wait_bar(bar(kKBarST), uint32_t(i) & 1u, ctl, p.status,
+                                            p.timeout_ns))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      tmem_ld32(tSt + lane_base + 32 * half, s);
+      tmem_ld32(tSt + lane_base + 64 + 32 * half, s + 32);
+      tmem_wait_ld();
+      // per query column -D and -L as pairs; block b covers queries
+      // [64 b + 32 half, +32). Pᵀ goes to Sᵀ columns [32 half + 16 b, +16),
+      // dSᵀ to [64 + 32 half + 16 b, +16): only columns this thread has read.
       const uint64_t* ndl = reinterpret_cast<const uint64_t*>(smem + stage(i) + 2 * kBTile);
-      uint32_t pw[32], dsw[32];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int cb = c0 + 32 * h;
-        float s[32], dp[32];
-        tmem_ld32(tSt + lane_base + cb, s);
-        tmem_ld32(tDPt + lane_base + cb, dp);
+      for (int b = 0; b < 2; ++b) {
+        const int cb = 64 * b + 32 * half;
         uint64_t nd2[16], nl2[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
           nd2[k] = ndl[cb / 2 + k];
           nl2[k] = ndl[64 + cb / 2 + k];
         }
-        tmem_wait_ld();
-        uint32_t(&po)[16] = *reinterpret_cast<uint32_t(*)[16]>(pw + 16 * h);
-        uint32_t(&dso)[16] = *reinterpret_cast<uint32_t(*)[16]>(dsw + 16 * h);
-        if (cls == SCA_TILE_FULL) ds_pairs<true>(s, dp, 0u, c2, nl2, nd2, dso, po);
-        else ds_pairs<false>(s, dp, vis[h], c2, nl2, nd2, dso, po);
+        const float(&sb)[32] = *reinterpret_cast<const float(*)[32]>(s + 32 * b);
+        const float(&dpb)[32] = *reinterpret_cast<const float(*)[32]>(dp + 32 * b);
+        uint32_t pw[16], dsw[16];
+        if (cls == SCA_TILE_FULL) ds_pairs<true>(sb, dpb, 0u, c2, nl2, nd2, dsw, pw);
+        else ds_pairs<false>(sb, dpb, vis[b], c2, nl2, nd2, dsw, pw);
+        tmem_st16(tSt + lane_base + 32 * half + 16 * b, pw);
+        tmem_st16(tSt + lane_base + 64 + 32 * half + 16 * b, dsw);
       }
-      tmem_st16(tSt + lane_base + c0, pw);  // Pᵀ over the first 32 columns of this half
-      tmem_st16(tSt + lane_base + c0 + 16, pw + 16);
-      tmem_st16(tDPt + lane_base + c0, dsw);  // dSᵀ likewise
-      tmem_st16(tDPt + lane_base + c0 + 16, dsw + 16);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kKBarDS));
