@@ -58,6 +58,7 @@ WORKLOADS["packed-360k-bwd"] = lambda: dataclasses.replace(W.packed_360k(), name
 BWD_WORKLOADS = {"packed-360k-bwd"}
 BWD_FLOP_FACTOR = 2.5   # five products per visible pair against the forward's two
 KERNEL_SOURCES = ["segment_causal_masked_b200/csrc/sca_kernels.cu",
+                  "segment_causal_masked_b200/csrc/sca_ptx.cuh",
                   "segment_causal_masked_b200/csrc/sca_internal.h"]
 
 
