@@ -51,11 +51,15 @@ WORKLOADS = {
     "480p-long-session-int8": lambda: dataclasses.replace(W.session_480p_long(),
                                                           name="480p-long-session-int8"),
 }
-INT8_WORKLOADS = {"480p-long-session-int8"}
+WORKLOADS["480p-single-turn-int8"] = lambda: dataclasses.replace(W.session_480p_single_turn(),
+                                                                 name="480p-single-turn-int8")
+INT8_WORKLOADS = {"480p-long-session-int8", "480p-single-turn-int8"}
 # the backward of the packed training batch (the forward that produces O and
 # LSE runs once, untimed; a step is one backward call)
 WORKLOADS["packed-360k-bwd"] = lambda: dataclasses.replace(W.packed_360k(), name="packed-360k-bwd")
-BWD_WORKLOADS = {"packed-360k-bwd"}
+WORKLOADS["packed-64k-bwd"] = lambda: dataclasses.replace(W.packed_360k(budget=64_000),
+                                                          name="packed-64k-bwd")
+BWD_WORKLOADS = {"packed-360k-bwd", "packed-64k-bwd"}
 BWD_FLOP_FACTOR = 2.5   # five products per visible pair against the forward's two
 KERNEL_SOURCES = ["segment_causal_masked_b200/csrc/sca_kernels.cu",
                   "segment_causal_masked_b200/csrc/sca_ptx.cuh",
