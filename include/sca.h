@@ -351,6 +351,16 @@ SCA_API int sca_action_causal_attn_bwd(const sca_metadata* md, int32_t heads, co
                                        uint64_t workspace_bytes, int32_t* dev_status,
                                        void* stream);
 
+/* Host view of the backward's key-major schedule (layouts without a cache;
+ * empty otherwise): kt_ptr[n_kv_tiles + 1] and kt_list[nnz], for each key tile
+ * the query tiles that see part of it in ascending order, each entry
+ * query tile | class << 24 (the transpose of the CSR schedule above);
+ * kt_order[n_kv_tiles], the key tiles most expensive first. Valid until the
+ * next build or destroy; all three are NULL for a layout with a cache. Any
+ * output may be NULL. */
+SCA_API int sca_metadata_get_bwd_schedule(const sca_metadata* md, const int32_t** kt_ptr,
+                                          const uint32_t** kt_list, const int32_t** kt_order);
+
 /* Workspace the backward needs: 2 · heads · round_up(n, 128) floats. */
 SCA_API int sca_attn_bwd_workspace_bytes(const sca_metadata* md, int32_t heads, uint64_t* bytes);
 

@@ -503,6 +503,16 @@ int sca_metadata_get_descriptors(const sca_metadata* md, const uint32_t** key_de
   return SCA_OK;
 }
 
+int sca_metadata_get_bwd_schedule(const sca_metadata* md, const int32_t** kt_ptr,
+                                  const uint32_t** kt_list, const int32_t** kt_order) {
+  if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
+  const bool has = !md->kt_ptr.empty();  // NULL outputs for a layout with a cache
+  if (kt_ptr) *kt_ptr = has ? md->kt_ptr.data() : nullptr;
+  if (kt_list) *kt_list = has ? md->kt_list.data() : nullptr;
+  if (kt_order) *kt_order = has ? md->kt_order.data() : nullptr;
+  return SCA_OK;
+}
+
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int sca_metadata_upload(sca_metadata* md, void* stream) {

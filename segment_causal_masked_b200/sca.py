@@ -33,6 +33,7 @@ EXPORTED = (
     "sca_metadata_create", "sca_build_segment_mask_metadata",
     "sca_build_segment_mask_metadata_ex", "sca_metadata_get_counts",
     "sca_metadata_get_schedule", "sca_metadata_get_descriptors", "sca_metadata_upload",
+    "sca_metadata_get_bwd_schedule",
     "sca_metadata_destroy", "sca_kv_cache_create", "sca_kv_cache_create_int8",
     "sca_kv_cache_append",
     "sca_kv_cache_truncate", "sca_kv_cache_get", "sca_kv_cache_destroy",
@@ -76,6 +77,9 @@ _SIGS = {
     "sca_metadata_get_counts": [_P, _pi64, _pi64, _pi64, _pi32, _pi32, _pi64, _pi64, _pi64],
     "sca_metadata_get_schedule": [_P, ctypes.POINTER(_pi32), ctypes.POINTER(_pi32),
                                   ctypes.POINTER(ctypes.POINTER(ctypes.c_uint8))],
+    "sca_metadata_get_bwd_schedule": [_P, ctypes.POINTER(_pi32),
+                                      ctypes.POINTER(ctypes.POINTER(ctypes.c_uint32)),
+                                      ctypes.POINTER(_pi32)],
     "sca_metadata_get_descriptors": [_P, ctypes.POINTER(ctypes.POINTER(ctypes.c_uint32)),
                                      ctypes.POINTER(ctypes.POINTER(ctypes.c_uint32))],
     "sca_metadata_upload": [_P, _P],
@@ -214,6 +218,24 @@ class Metadata:
         kv = np.ctypeslib.as_array(kt, shape=(max(n, 1),))[:n].copy()
         flag = np.ctypeslib.as_array(fl, shape=(max(n, 1),))[:n].copy()
         return row_ptr, kv, flag
+
+    def bwd_schedule(self):
+        """(kt_ptr, kt_list, kt_order) of the backward's key-major schedule as
+        numpy copies (empty arrays for a layout with a cache)."""
+        import numpy as np
+        c = self.counts()
+        kp, ko = _pi32(), _pi32()
+        kl = ctypes.POINTER(ctypes.c_uint32)()
+        _check(_lib.sca_metadata_get_bwd_schedule(self.handle, ctypes.byref(kp), ctypes.byref(kl),
+                                                  ctypes.byref(ko)))
+        if not kp:
+            return np.zeros(0, np.int32), np.zeros(0, np.uint32), np.zeros(0, np.int32)
+        n_kt = c["n_kv_tiles"]
+        kt_ptr = np.ctypeslib.as_array(kp, shape=(n_kt + 1,)).copy()
+        nnz = int(kt_ptr[-1])
+        kt_list = np.ctypeslib.as_array(kl, shape=(max(nnz, 1),))[:nnz].copy()
+        kt_order = np.ctypeslib.as_array(ko, shape=(n_kt,)).copy()
+        return kt_ptr, kt_list, kt_order
 
     def descriptors(self):
         """(key descriptors of the current keys [n], query descriptors [n, 2])."""

@@ -197,3 +197,30 @@ def test_int8_cache_handle_checks():
     assert e.value.code == sca.ERR_MISALIGNED
     c = sca.kv_cache_create_int8(2, 8, base, base, base, base, base)
     assert c.int8 and c.get() == (0, 0)
+
+
+@pytest.mark.parametrize("p", [W.tiny_packed(), W.small_packed(), W.small_packed(seed=21, n_segments=14),
+                               W.with_random_blocks(W.small_packed(seed=21, n_segments=14), 0.3, 9)],
+                         ids=lambda p: p.name)
+def test_backward_schedule_is_the_transposed_oracle_schedule(p):
+    """The backward's key-major lists: for every key tile, the query tiles
+    whose oracle class is not EMPTY, ascending, with that class; the order
+    is a permutation of the key tiles."""
+    lay = orule.Layout.of(p)
+    md = _builder(p)
+    kt_ptr, kt_list, kt_order = md.bwd_schedule()
+    row_ptr, kv, flag = osched.schedule(lay)
+    n_kt = md.counts()["n_kv_tiles"]
+    expect = [[] for _ in range(n_kt)]
+    for qt in range(len(row_ptr) - 1):
+        for i in range(row_ptr[qt], row_ptr[qt + 1]):
+            expect[int(kv[i])].append(qt | (int(flag[i]) << 24))
+    assert kt_ptr[0] == 0 and len(kt_ptr) == n_kt + 1
+    for t in range(n_kt):
+        assert kt_list[kt_ptr[t]:kt_ptr[t + 1]].tolist() == expect[t], t
+    assert sorted(kt_order.tolist()) == list(range(n_kt))
+
+
+def test_backward_schedule_absent_with_a_cache():
+    kt_ptr, kt_list, kt_order = _builder(W.small_session()).bwd_schedule()
+    assert len(kt_ptr) == 0 and len(kt_list) == 0 and len(kt_order) == 0
