@@ -342,16 +342,19 @@ class Session:
                                device=dev)
         torch.cuda.synchronize()
 
-    def step_backward(self, q=None, k=None, v=None, o=None, lse=None, d_o=None, ev=None):
-        """One backward call; `ev` = (start, end) events around it."""
+    def step_backward(self, q=None, k=None, v=None, o=None, lse=None, d_o=None, grads=None,
+                      ev=None):
+        """One backward call; `grads` = (dq, dk, dv) outputs (the session's by
+        default); `ev` = (start, end) events around it."""
         sca, p = self.sca, self.p
         s = self.stream.cuda_stream
+        dq, dk, dv = grads if grads is not None else (self.dq, self.dk, self.dv)
         if ev is not None:
             ev[0].record(self.stream)
         sca.action_causal_attn_bwd(self.md, p.heads, self.q if q is None else q,
                                    self.k_cur if k is None else k, self.v_cur if v is None else v,
                                    self.o if o is None else o, self.lse if lse is None else lse,
-                                   self.d_o if d_o is None else d_o, self.dq, self.dk, self.dv,
+                                   self.d_o if d_o is None else d_o, dq, dk, dv,
                                    p.softmax_scale, self.bws, None, self.status, s)
         if ev is not None:
             ev[1].record(self.stream)
@@ -440,47 +443,73 @@ def run_native(args, problem):
     ms_step = ms_total / args.steps
     value = whole_job_tflops(world, flops, args.steps, ms_total)
 
-    # ---- end to end through the API with pinned host buffers
+    # ---- end to end through the API with pinned host buffers. Every step
+    # uploads its inputs from pinned host memory and downloads its result;
+    # with two device copies of the inputs and outputs, step i+1's uploads
+    # (one stream) and step i's download (another) overlap step i's compute,
+    # as a serving loop would run. All of it lies inside the timed region.
     nq, h = problem.n_query_tokens, problem.heads
     pin = dict(pin_memory=True, dtype=torch.bfloat16)
-    hq = sess.q.cpu().pin_memory()
-    hk = sess.k_cur.cpu().pin_memory()
-    hv = sess.v_cur.cpu().pin_memory()
-    ho = torch.empty(nq, h, 128, **pin)
-    dq, dk, dv = torch.empty_like(sess.q), torch.empty_like(sess.k_cur), torch.empty_like(sess.v_cur)
+    if bwd:   # inputs q, k, v, o, lse, dO; results dq, dk, dv
+        host_in = [t.cpu().pin_memory() for t in (sess.q, sess.k_cur, sess.v_cur, sess.o, sess.lse,
+                                                  sess.d_o)]
+        host_out = [torch.empty(nq, h, 128, **pin) for _ in range(3)]
 
-    def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        sess.step(q=dq, k_cur=dk, v_cur=dv)
-        ho.copy_(sess.o, non_blocking=True)
+        def run(ins, outs):
+            q, k, v, o, lse, d_o = ins
+            sess.step_backward(q=q, k=k, v=v, o=o, lse=lse, d_o=d_o, grads=outs)
+    else:     # inputs q, k_cur, v_cur; result o
+        host_in = [t.cpu().pin_memory() for t in (sess.q, sess.k_cur, sess.v_cur)]
+        host_out = [torch.empty(nq, h, 128, **pin)]
 
-    bytes_in = 3 * hq.numel() * hq.element_size()
-    bytes_out = ho.numel() * ho.element_size()
-    if bwd:  # inputs q, k, v, o, lse, dO in; dq, dk, dv out
-        h_o, h_do, h_lse = sess.o.cpu().pin_memory(), sess.d_o.cpu().pin_memory(), sess.lse.cpu().pin_memory()
-        d_o_, d_do, d_lse = torch.empty_like(sess.o), torch.empty_like(sess.d_o), torch.empty_like(sess.lse)
-        h_g = [torch.empty(nq, h, 128, **pin) for _ in range(3)]
+        def run(ins, outs):
+            sess.step(q=ins[0], k_cur=ins[1], v_cur=ins[2], o=outs[0])
+    dev_in = [[torch.empty_like(t, device="cuda") for t in host_in] for _ in range(2)]
+    dev_out = [[torch.empty_like(t, device="cuda") for t in host_out] for _ in range(2)]
+    bytes_in = sum(t.numel() * t.element_size() for t in host_in)
+    bytes_out = sum(t.numel() * t.element_size() for t in host_out)
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()  # noqa: E731
+    in_ready, out_ready, out_read = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    used = [None, None]   # event after the compute that last read input set b
 
-        def e2e_step():  # noqa: F811
-            for dst, src in ((dq, hq), (dk, hk), (dv, hv), (d_o_, h_o), (d_do, h_do), (d_lse, h_lse)):
+    def upload(i):
+        b = i % 2
+        with torch.cuda.stream(h2d):
+            if used[b] is not None:
+                h2d.wait_event(used[b])
+            for dst, src in zip(dev_in[b], host_in):
                 dst.copy_(src, non_blocking=True)
-            sess.step_backward(q=dq, k=dk, v=dv, o=d_o_, lse=d_lse, d_o=d_do)
-            for dst, src in zip(h_g, (sess.dq, sess.dk, sess.dv)):
-                dst.copy_(src, non_blocking=True)
+            in_ready[b].record(h2d)
 
-        bytes_in = 5 * hq.numel() * hq.element_size() + h_lse.numel() * 4
-        bytes_out = 3 * hq.numel() * hq.element_size()
+    def e2e_steps(n):
+        upload(0)
+        for i in range(n):
+            b = i % 2
+            if i + 1 < n:
+                upload(i + 1)
+            sess.stream.wait_event(in_ready[b])
+            sess.stream.wait_event(out_read[b])
+            run(dev_in[b], dev_out[b])
+            used[b] = ev()
+            used[b].record(sess.stream)
+            out_ready[b].record(sess.stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(out_ready[b])
+                for dst, src in zip(host_out, dev_out[b]):
+                    dst.copy_(src, non_blocking=True)
+                out_read[b].record(d2h)
+        last = ev()
+        last.record(d2h)
+        sess.stream.wait_event(last)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    e2e_steps(args.warmup)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     e0.record(sess.stream)
-    for _ in range(args.steps):
-        e2e_step()
+    h2d.wait_event(e0)
+    e2e_steps(args.steps)
     e1.record(sess.stream)
     torch.cuda.synchronize()
     barrier()
