@@ -290,7 +290,7 @@ class Session:
         bf = torch.bfloat16
         self.desc = torch.zeros((self.capacity + 127) // 128 * 128, dtype=torch.int32, device=dev)
         if int8:
-            self.k_buf = torch.empty(h, self.capacity, 128, dtype=torch.int8, device=dev)
+            self.k_buf = torch.empty(h, self.capacity, 128, dtype=torch.uint8, device=dev)
             self.v_buf = torch.empty_like(self.k_buf)
             self.k_scale = torch.empty(h, self.capacity, dtype=torch.float32, device=dev)
             self.v_scale = torch.empty_like(self.k_scale)

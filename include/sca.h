@@ -210,7 +210,8 @@ SCA_API int sca_kv_cache_create(sca_kv_cache** out, int32_t heads, int32_t head_
  *     scale = max_d |x_d| / 127,   code_d = round_half_even(x_d / scale)
  * in fp32 from the bf16 values (a zero row: scale 0, codes 0), clamped to
  * [-127, 127]; the cached value is code * scale. Caller-owned buffers:
- *   k_codes, v_codes: int8 (two's complement) [heads][capacity][128];
+ *   k_codes, v_codes: uint8 [heads][capacity][128], each code stored
+ *                     offset-binary as code + 128 (1 ... 255);
  *   k_scale, v_scale: fp32 [heads][capacity];
  *   desc_buf:         uint32 [round_up(capacity, 128)] as above.
  * capacity must be a multiple of 4 (the scale rows are read with 16-byte

@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const AppendArgs a) {
 // two bf16 pairs): scale = max|x| / 127 and code = rint(x / scale) in fp32,
 // both divisions correctly rounded and the rounding to nearest even, codes
 // clamped to [-127, 127]; a zero row gets scale 0 and codes 0. Returns the
-// lane's four codes packed low byte first.
+// lane's four codes as offset-binary bytes (code + 128), low byte first.
 __device__ __forceinline__ uint32_t quantize_lane(uint2 raw, float& scale) {
   float x[4];
   x[0] = __uint_as_float(raw.x << 16);
@@ -93,12 +93,13 @@ __device__ __forceinline__ uint32_t quantize_lane(uint2 raw, float& scale) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
   scale = __fdiv_rn(amax, 127.f);
-  uint32_t packed = 0;
+  uint32_t packed = 0x80808080u;  // code 0 in every byte
   if (scale > 0.f) {
+    packed = 0u;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int qi = min(max(__float2int_rn(__fdiv_rn(x[i], scale)), -127), 127);
-      packed |= (uint32_t(qi) & 255u) << (8 * i);
+      packed |= uint32_t(qi + 128) << (8 * i);
     }
   }
   return packed;
@@ -176,8 +177,8 @@ __device__ __forceinline__ void exp_pack_store(const float (&x)[128], uint64_t s
   }
 }
 
-// INT8 cache: dequantise row r of a staged code tile (128 rows of 128 int8
-// codes, 128-byte swizzle, as the tensor copy lays it out) into row r of a
+// INT8 cache: dequantise row r of a staged code tile (128 rows of 128
+// offset-binary codes, 128-byte swizzle, as the tensor copy lays it out) into row r of a
 // bf16 operand tile in the layout the tensor copy of a bf16 tile gives (two
 // 64-column halves 16 KB apart, 128-byte swizzle). A code c becomes the exact
 // float c through the bit pattern 2^23 + (c + 128), then c * scale is rounded
@@ -195,7 +196,7 @@ __device__ __forceinline__ void dequant_row(const uint8_t* codes, float scale, u
     uint32_t out[8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const uint32_t u = words[k] ^ 0x80808080u;  // c + 128 in every byte
+      const uint32_t u = words[k];  // c + 128 in every byte (offset binary)
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         const float f0 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7540u + 2u * b));

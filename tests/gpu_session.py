@@ -30,7 +30,8 @@ class GpuSession:
         cap_pad = (self.capacity + 127) // 128 * 128
         self.desc = torch.zeros(cap_pad, dtype=torch.int32, device=self.dev)
         if int8:
-            self.k_buf = torch.zeros(h, self.capacity, 128, dtype=torch.int8, device=self.dev)
+            # codes are stored offset-binary (code + 128)
+            self.k_buf = torch.zeros(h, self.capacity, 128, dtype=torch.uint8, device=self.dev)
             self.v_buf = torch.zeros_like(self.k_buf)
             self.k_scale = torch.zeros(h, self.capacity, dtype=torch.float32, device=self.dev)
             self.v_scale = torch.zeros_like(self.k_scale)

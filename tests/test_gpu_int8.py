@@ -57,12 +57,12 @@ def test_append_codes_and_scales_bit_exact():
     nc = p.n_cache_tokens
     for buf, sc, name in ((s.k_buf, s.k_scale, "cache_k"), (s.v_buf, s.v_scale, "cache_v")):
         q_ref, s_ref = ocache.quantize_rows(inputs[name].float().numpy())   # [n, H, 128], [n, H]
-        codes = buf[:, :nc].cpu().numpy().transpose(1, 0, 2)
+        codes = buf[:, :nc].cpu().numpy().transpose(1, 0, 2).astype(np.int16) - 128  # offset binary
         scales = sc[:, :nc].cpu().numpy().T
         assert np.array_equal(codes, q_ref), name
         assert np.array_equal(scales.view(np.uint32), s_ref.view(np.uint32)), name
         assert not buf[:, nc:].any() and not sc[:, nc:].any()   # rows past the length untouched
-    k_codes = s.k_buf.cpu().numpy()
+    k_codes = s.k_buf.cpu().numpy().astype(np.int16) - 128
     assert not k_codes[0, 0].any() and s.k_scale[0, 0].item() == 0.0
     assert k_codes[0, 4, :3].tolist() == [127, 2, -4] and s.k_scale[0, 4].item() == 1.0
 
