@@ -53,7 +53,12 @@ WORKLOADS = {
 }
 WORKLOADS["480p-single-turn-int8"] = lambda: dataclasses.replace(W.session_480p_single_turn(),
                                                                  name="480p-single-turn-int8")
-INT8_WORKLOADS = {"480p-long-session-int8", "480p-single-turn-int8"}
+# the INT8 cache with a workspace that also holds a bf16 copy of it: the call
+# dequantises once (an HBM-bound copy) and runs the bf16 kernel on the copy
+WORKLOADS["480p-long-session-int8-copy"] = lambda: dataclasses.replace(
+    W.session_480p_long(), name="480p-long-session-int8-copy")
+INT8_WORKLOADS = {"480p-long-session-int8", "480p-single-turn-int8", "480p-long-session-int8-copy"}
+INT8_COPY_WORKLOADS = {"480p-long-session-int8-copy"}
 # the backward of the packed training batch (the forward that produces O and
 # LSE runs once, untimed; a step is one backward call)
 WORKLOADS["packed-360k-bwd"] = lambda: dataclasses.replace(W.packed_360k(), name="packed-360k-bwd")
@@ -275,7 +280,7 @@ class Session:
     """One replica of the workload on the current device: a cache holding the
     prior segments, the current segment's Q/K/V, outputs and metadata."""
 
-    def __init__(self, problem, seed: int, int8: bool = False):
+    def __init__(self, problem, seed: int, int8: bool = False, int8_copy: bool = False):
         import torch
 
         from segment_causal_masked_b200 import sca
@@ -318,6 +323,9 @@ class Session:
         self.md = sca.build_for(problem)
         ws_bytes = sca.attn_workspace_bytes(self.md, h)
         self.splits = ws_bytes > 0
+        if int8_copy:   # room for the bf16 copy of the INT8 cache after the split scratch
+            ws_bytes = (ws_bytes + 255) // 256 * 256 + sca.attn_int8_scratch_bytes(self.md, h)
+        self.int8_copy = int8_copy
         self.plan = sca.attn_plan(self.md, h)
         self.workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
         self.stream = torch.cuda.current_stream()
@@ -405,7 +413,8 @@ def run_native(args, problem):
 
     int8 = args.workload in INT8_WORKLOADS
     bwd = args.workload in BWD_WORKLOADS
-    sess = Session(problem, seed=1000 * 2 + rank, int8=int8)
+    int8_copy = args.workload in INT8_COPY_WORKLOADS
+    sess = Session(problem, seed=1000 * 2 + rank, int8=int8, int8_copy=int8_copy)
     from segment_causal_masked_b200 import sca
     sca_md = sca.build_for(problem)
     counts = sca_md.counts()
@@ -536,7 +545,9 @@ def run_native(args, problem):
                                 if sess.appends else "metadata build+upload, attention forward"),
                        "flop_count": ("10·d·H·A (five products per visible pair)" if bwd
                                       else "4·d·H·A (two products per visible pair)"),
-                       "kv_cache": "int8 codes + fp32 row scales" if int8 else "bf16",
+                       "kv_cache": ("int8 codes + fp32 row scales" + (", dequantised once per call"
+                                    " into a bf16 copy in the workspace" if int8_copy else
+                                    ", dequantised tile by tile in the kernel")) if int8 else "bf16",
                        "l2": "inputs larger than L2 (cached K/V %.2f GB per tensor)"
                              % (problem.n_cache_tokens * h * (132 if int8 else 256) / 1e9),
                        "parallelism": f"replicas x{world}",
@@ -549,7 +560,8 @@ def run_native(args, problem):
                          "peak_source": f"{peaks['source']} bf16 dense (burst)"},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": bytes_in,
                     "d2h_bytes_per_step": bytes_out, "ms_per_step": e2e_ms / args.steps},
-            "gpu_launches": (3 if bwd else 1 + int(sess.appends) + int(sess.splits)) * args.steps,
+            "gpu_launches": (3 if bwd else 1 + int(sess.appends) + int(sess.splits)
+                             + int(int8_copy)) * args.steps,
             "clocks": clock_info,
         }
         if not args.no_cpu_baseline:

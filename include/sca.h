@@ -280,6 +280,18 @@ SCA_API int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_meta
  * (0 when the plan splits nothing). */
 SCA_API int sca_attn_workspace_bytes(const sca_metadata* md, int32_t heads, uint64_t* bytes);
 
+/* INT8 cache: extra workspace for a bf16 copy of the cached K and V
+ * (2 · heads · n_cache · 256 bytes, each half 256-byte aligned). When the
+ * workspace given to the attention holds sca_attn_workspace_bytes (rounded up
+ * to 256) plus this, the call first dequantises the cache into it, once,
+ * with an HBM-bound copy kernel, and runs the bf16 kernel on the copy;
+ * otherwise the INT8 kernel dequantises tile by tile in shared memory, again
+ * for every query-tile pair that reads the tile. Both paths feed the same
+ * bf16 values to the products and give the same result bit for bit; the
+ * persistent cache stays INT8 either way (a model's per-layer caches can
+ * share one copy buffer). */
+SCA_API int sca_attn_int8_scratch_bytes(const sca_metadata* md, int32_t heads, uint64_t* bytes);
+
 /* The plan the next attention call with enough workspace would run: the
  * first n_full work items (query-tile pair x head) whole, the remaining
  * n_split items cut into `chunks` key ranges each. Any output may be NULL. */

@@ -897,6 +897,14 @@ int sca_attn_workspace_bytes(const sca_metadata* md, int32_t heads, uint64_t* by
   return SCA_OK;
 }
 
+int sca_attn_int8_scratch_bytes(const sca_metadata* md, int32_t heads, uint64_t* bytes) {
+  if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
+  if (heads < 1 || !bytes) return fail(SCA_ERR_INVALID_ARG, "need heads >= 1 and an output pointer");
+  // bf16 K and V of every cached key, each 256-byte aligned
+  *bytes = 2 * align_up(uint64_t(heads) * uint64_t(md->n_cache) * SCA_HEAD_DIM * 2, 256);
+  return SCA_OK;
+}
+
 int sca_attn_plan(const sca_metadata* md, int32_t heads, int32_t* n_full, int32_t* n_split,
                   int32_t* chunks) {
   if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
@@ -946,8 +954,36 @@ int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md
   int rc = make_map(&maps.q, q, uint64_t(heads), uint64_t(md->n_q), SCA_HEAD_DIM * 2, row, 1, SCA_TILE);
   if (!rc) rc = make_map(&maps.k_cur, k_cur, uint64_t(heads), uint64_t(md->n_q), SCA_HEAD_DIM * 2, row, 1, SCA_TILE);
   if (!rc) rc = make_map(&maps.v_cur, v_cur, uint64_t(heads), uint64_t(md->n_q), SCA_HEAD_DIM * 2, row, 1, SCA_TILE);
-  const bool int8_cache = md->n_cache > 0 && cache->int8;
-  if (!rc && int8_cache) {
+  bool int8_cache = md->n_cache > 0 && cache->int8;
+  // An INT8 cache with room for a bf16 copy of it after the split scratch:
+  // dequantise once here and run the bf16 kernel on the copy (the same
+  // values reach the products as in the kernel that dequantises tile by tile).
+  plan_for(md, heads, dev);
+  uint64_t scratch = 0;
+  if (int8_cache) sca_attn_int8_scratch_bytes(md, heads, &scratch);
+  const uint64_t split_ws = align_up(md->plan_ws, 256);
+  const bool via_scratch = int8_cache && workspace && workspace_bytes >= split_ws + scratch;
+  if (!rc && via_scratch) {
+    uint8_t* base = static_cast<uint8_t*>(workspace) + split_ws;
+    DequantArgs dq{};
+    dq.k_codes = cache->k;
+    dq.v_codes = cache->v;
+    dq.k_scale = cache->k_scale;
+    dq.v_scale = cache->v_scale;
+    dq.k_out = base;
+    dq.v_out = base + scratch / 2;
+    dq.n = md->n_cache;
+    dq.capacity = cache->capacity;
+    dq.heads = heads;
+    if (int rc2 = check_cuda(launch_dequant(dq, static_cast<cudaStream_t>(stream)), "dequant launch"))
+      return rc2;
+    const uint64_t hstride = uint64_t(md->n_cache) * SCA_HEAD_DIM * 2;
+    rc = make_map(&maps.k_cache, dq.k_out, uint64_t(md->n_cache), uint64_t(heads), SCA_HEAD_DIM * 2,
+                  hstride, SCA_TILE, 1);
+    if (!rc) rc = make_map(&maps.v_cache, dq.v_out, uint64_t(md->n_cache), uint64_t(heads),
+                           SCA_HEAD_DIM * 2, hstride, SCA_TILE, 1);
+    int8_cache = false;  // the bf16 kernel reads the copy
+  } else if (!rc && int8_cache) {
     const uint64_t n = uint64_t(md->n_cache), cap = uint64_t(cache->capacity);
     rc = make_code_map(&maps.k_cache, cache->k, n, uint64_t(heads), cap);
     if (!rc) rc = make_code_map(&maps.v_cache, cache->v, n, uint64_t(heads), cap);
@@ -962,7 +998,6 @@ int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md
   }
   if (rc) return rc;
 
-  plan_for(md, heads, dev);
   const uint8_t* d = static_cast<const uint8_t*>(md->dev);
   AttnArgs a{};
   a.qdesc = reinterpret_cast<const uint2*>(d + md->off_qdesc);

@@ -121,6 +121,20 @@ struct AppendArgs {
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
 
+// INT8 cache rows [0, n) of every head -> bf16 [heads][n][128].
+struct DequantArgs {
+  const void* k_codes;
+  const void* v_codes;
+  const float* k_scale;
+  const float* v_scale;
+  void* k_out;
+  void* v_out;
+  int64_t n;
+  int64_t capacity;
+  int32_t heads;
+};
+cudaError_t launch_dequant(const DequantArgs& a, cudaStream_t stream);
+
 // Attention backward (layouts without cached segments: keys = queries = the
 // n current tokens). Work-list views of the metadata, the workspace and the
 // tensors of one call.

@@ -133,6 +133,59 @@ __global__ void __launch_bounds__(256) kv_append_int8_kernel(const AppendArgs a)
   append_descriptors(a);
 }
 
+// INT8 cache -> bf16 copy [heads][n][128] (the scratch path of the
+// attention): each thread turns 16 codes of one row into bf16 with the
+// arithmetic of the attention kernel's own dequantisation (exact c from the
+// pattern 2^23 + (c + 128), c * scale rounded to fp32, then to bf16), so both
+// paths feed the products the same values bit for bit.
+__global__ void __launch_bounds__(256) kv_dequant_kernel(const DequantArgs a) {
+  const uint4* __restrict__ codes[2] = {static_cast<const uint4*>(a.k_codes),
+                                        static_cast<const uint4*>(a.v_codes)};
+  const float* __restrict__ scales[2] = {a.k_scale, a.v_scale};
+  uint4* __restrict__ outs[2] = {static_cast<uint4*>(a.k_out), static_cast<uint4*>(a.v_out)};
+  const int64_t per_tensor = int64_t(a.heads) * a.n * 8;  // 16-code chunks
+  const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+  const uint64_t off2 = f2(-8388736.f, -8388736.f);       // -(2^23 + 128)
+  const uint64_t zero2 = f2(0.f, 0.f);
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < 2 * per_tensor; i += stride) {
+    const int t = i >= per_tensor;
+    const int64_t c = i - t * per_tensor;                  // chunk within the tensor
+    const int64_t row = c >> 3;                            // head * n + token
+    const int64_t h = row / a.n, tok = row - h * a.n;
+    const int64_t src_row = h * a.capacity + tok;
+    const float s = scales[t][src_row];
+    const uint64_t s2 = f2(s, s);
+    const uint4 w = __ldg(codes[t] + src_row * 8 + (c & 7));
+    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+    uint32_t out[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const float f0 = __uint_as_float(__byte_perm(words[k], 0x4B000000u, 0x7540u + 2u * b));
+        const float f1 = __uint_as_float(__byte_perm(words[k], 0x4B000000u, 0x7541u + 2u * b));
+        float v0, v1;
+        unf2(fma2(add2(f2(f0, f1), off2), s2, zero2), v0, v1);
+        out[2 * k + b] = pack_bf16(v0, v1);
+      }
+    }
+    outs[t][c * 2] = make_uint4(out[0], out[1], out[2], out[3]);
+    outs[t][c * 2 + 1] = make_uint4(out[4], out[5], out[6], out[7]);
+  }
+}
+
+cudaError_t launch_dequant(const DequantArgs& a, cudaStream_t stream) {
+  if (a.n <= 0) return cudaSuccess;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t work = 2 * int64_t(a.heads) * a.n * 8;
+  int64_t blocks = (work + 255) / 256;
+  blocks = blocks < int64_t(sms) * 8 ? blocks : int64_t(sms) * 8;
+  kv_dequant_kernel<<<unsigned(blocks), 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
   if (a.n <= 0) return cudaSuccess;
   int dev = 0, sms = 148;
@@ -615,12 +668,13 @@ __global__ void __launch_bounds__(threads_for(kInt8), 1)
         const float mx = max3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
         // The running max only moves when it grows by more than the threshold
         // (exact: l and O share the stale max until the final division).
-        const float m_cand = mx * p.scale_log2;
+        // rounded on its own (no FMA with the subtraction below), so that
+        // every instantiation of this kernel takes the same alpha
+        const float m_cand = __fmul_rn(mx, p.scale_log2);
         const bool grow = m_cand > m_run + kRescaleThreshold;
         const bool rescale = grow && m_run != -INFINITY && o_init;
         const float alpha = rescale ? ex2(m_run - m_cand) : 1.f;
         if (grow) m_run = m_cand;
-        l_run *= alpha;
         const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
         const uint64_t negm2 = f2(neg_m, neg_m);
         uint64_t acc[2] = {0ull, 0ull};  // packed partial sums
@@ -634,7 +688,9 @@ __global__ void __launch_bounds__(threads_for(kInt8), 1)
         }
         float a0, a1;
         unf2(add2(acc[0], acc[1]), a0, a1);
-        l_run += a0 + a1;
+        // one explicit rounding (l alpha + sum), so every instantiation of
+        // this kernel gives the same l, whatever the compiler would contract
+        l_run = fmaf(l_run, alpha, a0 + a1);
         // Rescale O. tcgen05.ld/st are warp-collective: the whole warp
         // rewrites O if any row needs it (alpha = 1 for the others). O of
         // earlier tiles was complete when S of this tile completed (in-order

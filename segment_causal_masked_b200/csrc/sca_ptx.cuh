@@ -261,11 +261,10 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float m;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
-  return m;
-}
+// Two 2-input maxima. (The 3-input max.f32 of sm_100 returned a wrong
+// finite value for three -inf inputs in one instantiation of the attention
+// kernel, where a row of masked scores must keep its running max at -inf.)
+__device__ __forceinline__ float max3(float a, float b, float c) { return fmaxf(fmaxf(a, b), c); }
 
 // Packed fp32 pairs (one instruction for two lanes of work on sm_100).
 __device__ __forceinline__ uint64_t f2(float a, float b) {

@@ -38,7 +38,7 @@ EXPORTED = (
     "sca_kv_cache_append",
     "sca_kv_cache_truncate", "sca_kv_cache_get", "sca_kv_cache_destroy",
     "sca_action_causal_attn_fwd", "sca_action_causal_attn_fwd_static_ws",
-    "sca_attn_workspace_bytes", "sca_attn_plan",
+    "sca_attn_workspace_bytes", "sca_attn_plan", "sca_attn_int8_scratch_bytes",
     "sca_action_causal_attn_bwd", "sca_attn_bwd_workspace_bytes",
     "sca_set_split_override",
     "sca_last_error", "sca_debug_bounded_wait", "sca_debug_exp2",
@@ -95,6 +95,7 @@ _SIGS = {
     "sca_action_causal_attn_fwd_static_ws": [_P, _P, _i32, _P, _P, _P, _P, _P, ctypes.c_float,
                                              _P, _P],
     "sca_attn_workspace_bytes": [_P, _i32, ctypes.POINTER(ctypes.c_uint64)],
+    "sca_attn_int8_scratch_bytes": [_P, _i32, ctypes.POINTER(ctypes.c_uint64)],
     "sca_action_causal_attn_bwd": [_P, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_float,
                                    _P, ctypes.c_uint64, _P, _P],
     "sca_attn_bwd_workspace_bytes": [_P, _i32, ctypes.POINTER(ctypes.c_uint64)],
@@ -396,6 +397,14 @@ def action_causal_attn_bwd(md: Metadata, heads: int, q, k, v, o, lse, d_o, dq, d
                                            _ptr(dv), float(softmax_scale), _ptr(workspace),
                                            int(workspace_bytes or 0), _ptr(dev_status),
                                            _stream(stream)))
+
+
+def attn_int8_scratch_bytes(md: Metadata, heads: int) -> int:
+    """Extra workspace that lets an INT8-cache attention dequantise once into
+    a bf16 copy (see include/sca.h)."""
+    b = ctypes.c_uint64()
+    _check(_lib.sca_attn_int8_scratch_bytes(md.handle, int(heads), ctypes.byref(b)))
+    return int(b.value)
 
 
 def attn_workspace_bytes(md: Metadata, heads: int) -> int:

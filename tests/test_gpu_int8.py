@@ -146,3 +146,37 @@ def test_int8_full_size_sampled_rows():
     o_ref, lse_ref = oattn.attention_rows(lay, q, k, v, rows, p.softmax_scale, heads=heads)
     compare(o[rows][:, heads], lse[heads][:, rows], o_ref, lse_ref)
     assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+
+
+def _fwd(s, p, ws_bytes):
+    o = torch.full((p.n_query_tokens, p.heads, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((p.heads, p.n_query_tokens), float("nan"), device="cuda")
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device="cuda")
+    sca.action_causal_attn_fwd(s.cache, s.md, p.heads, s.q, s.k_cur, s.v_cur, o, lse,
+                               p.softmax_scale, ws, ws_bytes, s.status)
+    torch.cuda.synchronize()
+    assert int(s.status.item()) == 0
+    return o, lse
+
+
+@pytest.mark.parametrize("chunks", [0, 3])
+@pytest.mark.parametrize("p", [W.small_session(heads=4), _multi_pair(),
+                               W.with_history(W.small_session(heads=2), 1)], ids=lambda p: p.name)
+def test_int8_scratch_path_equals_tile_path(p, chunks):
+    """With room for a bf16 copy of the cache, the call dequantises once and
+    runs the bf16 kernel: the same values reach the products, so the result
+    equals the tile-by-tile INT8 kernel's bit for bit; it matches the oracle."""
+    s = GpuSession(p, W.make_inputs(p, 77, 3.0), int8=True)
+    try:
+        sca.set_split_override(chunks)
+        split = (sca.attn_workspace_bytes(s.md, p.heads) + 255) // 256 * 256
+        scratch = sca.attn_int8_scratch_bytes(s.md, p.heads)
+        assert scratch == 2 * ((p.heads * p.n_cache_tokens * 256 + 255) // 256 * 256)
+        o1, l1 = _fwd(s, p, split)               # tile by tile
+        o2, l2 = _fwd(s, p, split + scratch)     # one bf16 copy first
+    finally:
+        sca.set_split_override(0)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)   # the same values reach the products
+    q, k, v = oracle_inputs(W.make_inputs(p, 77, 3.0), int8=True)
+    o_ref, lse_ref = oattn.attention(orule.Layout.of(p), q, k, v, p.softmax_scale)
+    compare(o2, l2, o_ref, lse_ref)
