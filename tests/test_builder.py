@@ -224,3 +224,25 @@ def test_backward_schedule_is_the_transposed_oracle_schedule(p):
 def test_backward_schedule_absent_with_a_cache():
     kt_ptr, kt_list, kt_order = _builder(W.small_session()).bwd_schedule()
     assert len(kt_ptr) == 0 and len(kt_list) == 0 and len(kt_order) == 0
+
+
+def test_backward_and_int8_copy_workspace_sizes():
+    """Host-only size queries: the backward's −D/−LSE rows per head padded to
+    whole tiles, and the INT8 copy of the cached K and V (two halves, each
+    256-byte aligned)."""
+    p = W.small_packed()
+    md = _builder(p)
+    n_pad = md.counts()["n_q_tiles"] * 128
+    assert sca.attn_bwd_workspace_bytes(md, 3) == 2 * 3 * n_pad * 4
+    s = _builder(W.small_session())
+    nc = W.small_session().n_cache_tokens
+    half = (5 * nc * 256 + 255) // 256 * 256
+    assert sca.attn_int8_scratch_bytes(s, 5) == 2 * half
+
+
+def test_backward_refuses_metadata_not_uploaded():
+    md = _builder(W.tiny_packed())
+    with pytest.raises(sca.ScaError) as e:
+        sca.action_causal_attn_bwd(md, 2, 16, 16, 16, 16, 16, 16, 16, 16, 16, workspace=256,
+                                   workspace_bytes=1 << 20, stream=0)
+    assert e.value.code == sca.ERR_INVALID_ARG and "uploaded" in str(e.value)
