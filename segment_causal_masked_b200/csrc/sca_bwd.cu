@@ -196,8 +196,12 @@ constexpr int kQKSlots = 3, kQVSlots = 2;
 constexpr uint32_t kQBarQD = 0, kQBarKF = 1, kQBarKE = kQBarKF + kQKSlots,
                    kQBarVF = kQBarKE + kQKSlots, kQBarVE = kQBarVF + kQVSlots,
                    kQBarS = kQBarVE + kQVSlots, kQBarDP = kQBarS + 2, kQBarDS = kQBarDP + 1,
-                   kQBarRD = kQBarDS + 1, kQBarDone = kQBarRD + 1, kQBarDrain = kQBarDone + 1,
+                   kQBarRD = kQBarDS + 2, kQBarDone = kQBarRD + 1, kQBarDrain = kQBarDone + 1,
                    kQNumBars = kQBarDrain + 1;
+// dS barriers alternate by step parity: the elementwise warps can finish step
+// j + 1 before the MMA thread has seen step j (the next dP starts on the
+// read-done signal), and a single barrier could then run two phases ahead
+// of the MMA thread's parity wait.
 constexpr uint32_t kQOffBar = 7 * kBTile;
 constexpr uint32_t kQOffCtl = kQOffBar + kQNumBars * 8;
 constexpr uint32_t kQOffSlot = kQOffCtl + 16;
@@ -242,6 +246,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     mbar_init(bar(kQBarS + 1), 1);
     mbar_init(bar(kQBarDP), 1);
     mbar_init(bar(kQBarDS), 256);
+    mbar_init(bar(kQBarDS + 1), 256);
     mbar_init(bar(kQBarRD), 256);
     mbar_init(bar(kQBarDone), 1);
     mbar_init(bar(kQBarDrain), 1);
@@ -358,7 +363,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
             mma_commit(bar(kQBarDP));
             mma_commit(bar(kQBarVE + (j + 1) % kQVSlots));
           }
-          if (!(ok = wait_bar(bar(kQBarDS), uint32_t(j) & 1u, ctl, p.status, p.timeout_ns))) break;
+          if (!(ok = wait_bar(bar(kQBarDS + (j & 1)), uint32_t(j >> 1) & 1u, ctl, p.status,
+                              p.timeout_ns)))
+            break;
           tc_fence_after();
           mma_ts8_split(tDQ, tSj, tSj + 64, desc_mnmajor(kslot(j)), kIdescPV, j > 0 ? 1u : 0u);
           mma_commit(bar(kQBarKE + j % kQKSlots));
@@ -437,7 +444,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
       tmem_st16(tSj + c0 + 16, dsw + 16);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(kQBarDS));
+      mbar_arrive(bar(kQBarDS + (j & 1)));
       ++j;
     }
     // epilogue: dQ row (this half) = scale * accumulated dS K
