@@ -1,0 +1,388 @@
+"""Model check of the kernels' mbarrier protocols (CPU, no GPU).
+
+Each pipeline of the CUDA kernels is restated here as roles (TMA producer,
+dequantiser, MMA issuer, elementwise/softmax warps) that wait on and arrive at
+barriers with the kernels' own slot and parity formulas. An mbarrier is a
+completed-phase counter; a parity wait succeeds when the phase with that
+parity has completed, which is only meaningful while the barrier is at most
+one phase away from the use the waiter expects. The simulation advances the
+roles in random interleavings and completes TMA copies in random order, and
+fails on: a deadlock, a slot refilled while its contents are still to be read,
+or a wait that sees its barrier two phases away.
+
+Pipelines: the attention forward's K/V ring with the INT8 cache's staged code
+slots (a prefix of cache tiles dequantised into the ring, then current tiles
+loaded directly), and the backward's dQ and dK/dV kernels.
+"""
+import random
+
+import pytest
+
+
+class Bar:
+    def __init__(self, count):
+        self.count, self.pending, self.completed, self.tx = count, count, 0, 0
+
+    def arrive(self, n=1):
+        self.pending -= n
+        assert self.pending >= 0, "more arrivals than the barrier's count"
+        self._check()
+
+    def expect(self, nbytes):  # arrive.expect_tx
+        self.tx += nbytes
+        self.arrive()
+
+    def complete_tx(self, nbytes):
+        self.tx -= nbytes
+        assert self.tx >= 0
+        self._check()
+
+    def _check(self):
+        if self.pending == 0 and self.tx == 0:
+            self.completed += 1
+            self.pending = self.count
+
+
+def wait(name, parity, use):
+    """Wait for use `use` (0-based) of barrier `name` to complete."""
+    return ("wait", name, parity, use)
+
+
+def run(roles, bars, seed):
+    rng = random.Random(seed)
+    waiting = {k: None for k in roles}
+    done, copies = set(), []
+    while len(done) < len(roles):
+        progressed = False
+        if copies and rng.random() < 0.5:
+            name, nbytes = copies.pop(rng.randrange(len(copies)))
+            bars[name].complete_tx(nbytes)
+            progressed = True
+        order = list(roles)
+        rng.shuffle(order)
+        for k in order:
+            if k in done:
+                continue
+            w = waiting[k]
+            if w is not None:
+                _, name, parity, use = w
+                b = bars[name]
+                if (b.completed & 1) != parity:
+                    assert b.completed == use + 1, (k, name, "barrier a phase ahead", b.completed, use)
+                    waiting[k] = None
+                else:
+                    assert b.completed == use, (k, name, "barrier a phase behind", b.completed, use)
+                    continue
+            try:
+                while True:
+                    ev = next(roles[k])
+                    if ev[0] == "wait":
+                        waiting[k] = ev
+                        break
+                    if ev[0] == "copy":
+                        copies.append((ev[1], ev[2]))
+                    if ev[0] == "work" and rng.random() < 0.3:
+                        break
+                progressed = True
+            except StopIteration:
+                done.add(k)
+                progressed = True
+        assert progressed or copies, ("deadlock", {k: waiting[k] for k in roles if k not in done})
+    assert not copies, "a copy still in flight when the CTA exits"
+
+
+# ---------------------------------------------------------------------------
+# attention forward, INT8 cache: ring of `ring` operand slots, `cslots` code
+# slots; iteration it = 2j (K of key tile j) or 2j + 1 (V)
+# ---------------------------------------------------------------------------
+
+def forward_int8(staged_tiles, ring, cslots, seed):
+    n = len(staged_tiles)
+    bars = {}
+    for s in range(ring):
+        bars[("full", s)] = Bar(128)
+        bars[("empty", s)] = Bar(1)
+    for s in range(cslots):
+        bars[("cfull", s)] = Bar(1)
+        bars[("cempty", s)] = Bar(128)
+    for t in range(2):
+        bars[("S", t)] = Bar(1)
+        bars[("P", t)] = Bar(1)
+        bars[("O", t)] = Bar(1)
+    ring_owner, code_owner = {}, {}
+    staged = lambda i: staged_tiles[i >> 1]  # noqa: E731
+
+    def producer():
+        for it in range(2 * n):
+            if staged(it):
+                cs = it % cslots
+                yield wait(("cempty", cs), ((it // cslots) & 1) ^ 1, it // cslots - 1)
+                assert code_owner.get(cs) is None
+                code_owner[cs] = it
+                bars[("cfull", cs)].expect(1)
+                yield ("copy", ("cfull", cs), 1)
+            else:
+                if it > 0 and staged(it - 1):  # wait for the whole staged prefix
+                    for i2 in range(max(0, it - cslots), it):
+                        yield wait(("cempty", i2 % cslots), (i2 // cslots) & 1, i2 // cslots)
+                s = it % ring
+                yield wait(("empty", s), ((it // ring) & 1) ^ 1, it // ring - 1)
+                assert ring_owner.get(s) is None, "ring slot refilled while in use"
+                ring_owner[s] = it
+                bars[("full", s)].expect(1)
+                bars[("full", s)].arrive(127)
+                yield ("copy", ("full", s), 1)
+
+    def dequantiser():
+        for it in range(2 * n):
+            if not staged(it):
+                break
+            cs, s = it % cslots, it % ring
+            yield wait(("cfull", cs), (it // cslots) & 1, it // cslots)
+            yield wait(("empty", s), ((it // ring) & 1) ^ 1, it // ring - 1)
+            assert code_owner.get(cs) == it and ring_owner.get(s) is None
+            ring_owner[s] = it
+            yield ("work",)
+            bars[("full", s)].arrive(128)
+            code_owner[cs] = None
+            bars[("cempty", cs)].arrive(128)
+
+    def mma():
+        def use(it):
+            assert ring_owner.get(it % ring) == it, "operand slot holds another tile"
+
+        def release(it):
+            use(it)
+            ring_owner[it % ring] = None
+            bars[("empty", it % ring)].arrive()
+
+        if n:
+            yield wait(("full", 0), 0, 0)
+            use(0)
+            bars[("S", 0)].arrive()
+            bars[("S", 1)].arrive()
+            release(0)
+        for j in range(n):
+            itv, itk = 2 * j + 1, 2 * j + 2
+            more = j + 1 < n
+            yield wait(("full", itv % ring), (itv // ring) & 1, itv // ring)
+            yield wait(("P", 0), j & 1, j)
+            use(itv)
+            if more:
+                yield wait(("full", itk % ring), (itk // ring) & 1, itk // ring)
+                use(itk)
+                bars[("S", 0)].arrive()
+            yield wait(("P", 1), j & 1, j)
+            release(itv)
+            if more:
+                bars[("S", 1)].arrive()
+                release(itk)
+        bars[("O", 0)].arrive()
+        bars[("O", 1)].arrive()
+
+    def softmax(t):
+        for j in range(n):
+            yield wait(("S", t), j & 1, j)
+            yield ("work",)
+            bars[("P", t)].arrive()
+        if n:
+            yield wait(("O", t), 0, 0)
+
+    run({"producer": producer(), "dequantiser": dequantiser(), "mma": mma(),
+         "softmax0": softmax(0), "softmax1": softmax(1)}, bars, seed)
+
+
+@pytest.mark.parametrize("ring, cslots", [(3, 4), (4, 2), (3, 3), (2, 5)])
+def test_forward_int8_pipeline(ring, cslots):
+    """The shipped INT8 depths (3 ring slots, 4 code slots) and others; every
+    prefix length of cache tiles, including none (the bf16 case) and all."""
+    for n in range(0, 9):
+        for n_staged in range(0, n + 1):
+            for seed in range(8):
+                forward_int8([True] * n_staged + [False] * (n - n_staged), ring, cslots, seed)
+
+
+# ---------------------------------------------------------------------------
+# backward: dQ (query-major) and dK/dV (key-major)
+# ---------------------------------------------------------------------------
+
+def backward_dq(n, seed, ks=3, vs=2):
+    bars = {("KF", s): Bar(1) for s in range(ks)}
+    bars.update({("KE", s): Bar(1) for s in range(ks)})
+    bars.update({("VF", s): Bar(1) for s in range(vs)})
+    bars.update({("VE", s): Bar(1) for s in range(vs)})
+    for name in ("QD", ("S", 0), ("S", 1), "DP", "DONE", ("DS", 0), ("DS", 1), "RD"):
+        bars[name] = Bar(1)
+    kslot, vslot, sbuf, dp = {}, {}, {}, {}
+
+    def producer():
+        bars["QD"].expect(1)
+        yield ("copy", "QD", 1)
+        for j in range(n):
+            yield wait(("KE", j % ks), ((j // ks) & 1) ^ 1, j // ks - 1)
+            assert kslot.get(j % ks) is None
+            kslot[j % ks] = j
+            bars[("KF", j % ks)].expect(1)
+            yield ("copy", ("KF", j % ks), 1)
+            yield wait(("VE", j % vs), ((j // vs) & 1) ^ 1, j // vs - 1)
+            assert vslot.get(j % vs) is None
+            vslot[j % vs] = j
+            bars[("VF", j % vs)].expect(1)
+            yield ("copy", ("VF", j % vs), 1)
+
+    def mma():
+        yield wait("QD", 0, 0)
+
+        def qk(j, buf):
+            assert kslot[j % ks] == j and sbuf.get(buf) in (None, "read")
+            sbuf[buf] = ("S", j)
+
+        if n:
+            yield wait(("KF", 0), 0, 0)
+            qk(0, 0)
+            bars[("S", 0)].arrive()
+            yield wait(("VF", 0), 0, 0)
+            dp["v"] = 0
+            bars["DP"].arrive()
+            vslot[0] = None
+            bars[("VE", 0)].arrive()
+            if n > 1:
+                yield wait(("KF", 1), 0, 0)
+                qk(1, 1)
+                bars[("S", 1)].arrive()
+        for j in range(n):
+            yield wait("RD", j & 1, j)
+            if j + 1 < n:
+                yield wait(("VF", (j + 1) % vs), ((j + 1) // vs) & 1, (j + 1) // vs)
+                assert vslot[(j + 1) % vs] == j + 1 and dp.get("read") == j
+                dp["v"] = j + 1
+                bars["DP"].arrive()
+                vslot[(j + 1) % vs] = None
+                bars[("VE", (j + 1) % vs)].arrive()
+            yield wait(("DS", j & 1), (j >> 1) & 1, j >> 1)
+            assert sbuf[j & 1] == ("dS", j) and kslot[j % ks] == j
+            sbuf[j & 1] = "read"
+            kslot[j % ks] = None
+            bars[("KE", j % ks)].arrive()
+            if j + 2 < n:
+                yield wait(("KF", (j + 2) % ks), ((j + 2) // ks) & 1, (j + 2) // ks)
+                qk(j + 2, j & 1)
+                bars[("S", j & 1)].arrive()
+        bars["DONE"].arrive()
+
+    def elementwise():
+        for j in range(n):
+            yield wait(("S", j & 1), (j >> 1) & 1, j >> 1)
+            yield wait("DP", j & 1, j)
+            assert sbuf[j & 1] == ("S", j) and dp["v"] == j
+            dp["read"] = j
+            bars["RD"].arrive()
+            yield ("work",)
+            sbuf[j & 1] = ("dS", j)
+            bars[("DS", j & 1)].arrive()
+        yield wait("DONE", 0, 0)
+
+    run({"producer": producer(), "mma": mma(), "elementwise": elementwise()}, bars, seed)
+
+
+def backward_dkdv(n, seed, stages=2):
+    bars = {("F", s): Bar(1) for s in range(stages)}
+    bars.update({("E", s): Bar(1) for s in range(stages)})
+    for name in ("KV", "ST", "DPT", "DONE", "RD", "DS"):
+        bars[name] = Bar(1)
+    stage, st, dpt = {}, {}, {}
+
+    def producer():
+        bars["KV"].expect(1)
+        yield ("copy", "KV", 1)
+        for i in range(n):
+            yield wait(("E", i % stages), ((i // stages) & 1) ^ 1, i // stages - 1)
+            assert stage.get(i % stages) is None
+            stage[i % stages] = i
+            bars[("F", i % stages)].expect(1)
+            yield ("copy", ("F", i % stages), 1)
+
+    def mma():
+        yield wait("KV", 0, 0)
+        if n:
+            yield wait(("F", 0), 0, 0)
+            st["v"] = ("S", 0)
+            bars["ST"].arrive()
+            dpt["v"] = 0
+            bars["DPT"].arrive()
+        for i in range(n):
+            yield wait("RD", i & 1, i)
+            if i + 1 < n:
+                yield wait(("F", (i + 1) % stages), ((i + 1) // stages) & 1, (i + 1) // stages)
+                assert stage[(i + 1) % stages] == i + 1 and dpt.get("read") == i
+                dpt["v"] = i + 1
+                bars["DPT"].arrive()
+            yield wait("DS", i & 1, i)
+            assert st["v"] == ("PdS", i) and stage[i % stages] == i
+            stage[i % stages] = None
+            bars[("E", i % stages)].arrive()
+            if i + 1 < n:
+                st["v"] = ("S", i + 1)
+                bars["ST"].arrive()
+        bars["DONE"].arrive()
+
+    def elementwise():
+        for i in range(n):
+            yield wait(("F", i % stages), (i // stages) & 1, i // stages)
+            yield wait("DPT", i & 1, i)
+            assert dpt["v"] == i
+            dpt["read"] = i
+            bars["RD"].arrive()
+            yield wait("ST", i & 1, i)
+            assert st["v"] == ("S", i) and stage[i % stages] == i
+            yield ("work",)
+            st["v"] = ("PdS", i)
+            bars["DS"].arrive()
+        yield wait("DONE", 0, 0)
+
+    run({"producer": producer(), "mma": mma(), "elementwise": elementwise()}, bars, seed)
+
+
+def test_backward_dq_pipeline():
+    for n in range(0, 12):
+        for seed in range(25):
+            backward_dq(n, seed)
+
+
+def test_backward_dkdv_pipeline():
+    for n in range(0, 12):
+        for seed in range(25):
+            backward_dkdv(n, seed)
+
+
+def test_single_ds_barrier_would_be_caught():
+    """The model check is sharp: with one dS barrier instead of two (the
+    dQ kernel before the fix), some interleaving lets the elementwise warps
+    run two phases ahead of the MMA thread's parity wait."""
+    import re
+    import inspect
+    src = inspect.getsource(backward_dq)
+    src = re.sub(r'\("DS", j & 1\), \(j >> 1\) & 1, j >> 1', '("DS", 0), j & 1, j', src)
+    src = src.replace('bars[("DS", j & 1)].arrive()', 'bars[("DS", 0)].arrive()')
+    scope = dict(globals())
+    exec(src, scope)
+    with pytest.raises(AssertionError):
+        for n in range(2, 8):
+            for seed in range(40):
+                scope["backward_dq"](n, seed)
+
+
+def test_missing_prefix_wait_would_be_caught():
+    """Likewise for the INT8 producer: without its wait for the staged prefix
+    before the first direct load, more code slots than ring slots let a
+    parity wait on a ring slot pass a phase early."""
+    import inspect
+    src = inspect.getsource(forward_int8)
+    src = src.replace("if it > 0 and staged(it - 1):", "if False:")
+    scope = dict(globals())
+    exec(src, scope)
+    with pytest.raises(AssertionError):
+        for n in range(2, 9):
+            for n_staged in range(1, n):
+                for seed in range(8):
+                    scope["forward_int8"]([True] * n_staged + [False] * (n - n_staged), 2, 5, seed)
