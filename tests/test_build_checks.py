@@ -1,4 +1,5 @@
-"""The build's launch-register check (CPU; nvcc cross-compiles for sm_100a).
+"""Build-level checks on the CPU: the launch-register check (nvcc
+cross-compiles for sm_100a) and a plain C program calling the library.
 
 The warp-specialised kernels regroup registers with setmaxnreg: some
 warpgroups grow, the others shrink, and the shares add up to the registers
@@ -6,7 +7,8 @@ the block was launched with. If ptxas gave a kernel fewer registers per
 thread than its split assumes, the growing warpgroups would wait forever on
 the GPU. The build reads ptxas's report and refuses such a library; these
 tests check that the report parser finds a mismatch and that the kernels as
-they stand pass.
+they stand pass. The last test compiles tests/c/abi_host_only.c with gcc
+against include/sca.h and libsca.so alone and runs its host-side calls.
 """
 import os
 import shutil
@@ -64,3 +66,38 @@ def test_current_kernels_get_the_registers_their_splits_need(tmp_path):
     with ThreadPoolExecutor(2) as ex:
         log = "".join(ex.map(compile_one, ["sca_kernels.cu", "sca_bwd.cu"]))
     B.check_launch_registers(log)
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+def test_plain_c_caller_of_the_abi(tmp_path):
+    """tests/c/abi_host_only.c uses nothing but include/sca.h and libsca.so:
+    it builds the 480p long session's metadata, reads counts and schedule,
+    and checks two refused layouts. A is the hand-worked closed form
+    12,090 (12 x 12,218 + 12,250) + 128 x 12,218 + 128 x 12,250; the tile
+    counts must equal what the Python binding reads from the same library."""
+    from segment_causal_masked_b200 import sca
+    from segment_causal_masked_b200 import workloads as W
+
+    exe = tmp_path / "abi_host_only"
+    lib_dir = os.path.dirname(sca.LIB_PATH)
+    src = os.path.join(os.path.dirname(os.path.abspath(__file__)), "c", "abi_host_only.c")
+    cc = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", B.INCLUDE, src,
+                         "-L", lib_dir, "-lsca", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, run.stdout + run.stderr
+    lines = dict(line.split(" ", 1) for line in run.stdout.strip().splitlines())
+
+    counts = [int(x) for x in lines["counts"].split()]
+    assert counts[0] == 12_090 * (12 * 12_218 + 12_250) + 128 * 12_218 + 128 * 12_250
+    c = sca.build_for(W.session_480p_long()).counts()
+    assert counts == [c["unmasked_pairs"], c["n_queries"], c["n_cache_keys"], c["n_q_tiles"],
+                      c["n_kv_tiles"], c["nnz"], c["n_full"], c["n_partial"]]
+    assert counts[1:5] == [12_346, 148_152, 97, 1158 + 97]
+    assert lines["schedule"].split() == [str(c["nnz"]), "0", str(sca.TILE_FULL)]
+
+    for key in ("bad_segment", "bad_window"):
+        code, message = lines[key].split(" ", 1)
+        assert int(code) == sca.ERR_INVALID_ARG and message, key
+    assert "num_frames" in lines["bad_segment"] and "[24, 32)" in lines["bad_window"]
