@@ -298,6 +298,14 @@ SCA_API int sca_attn_int8_scratch_bytes(const sca_metadata* md, int32_t heads, u
 SCA_API int sca_attn_plan(const sca_metadata* md, int32_t heads, int32_t* n_full,
                           int32_t* n_split, int32_t* chunks);
 
+/* The plan (and its workspace bytes) for a device with `sms` SMs, without
+ * touching any device: for planning ahead of a launch on another GPU, and
+ * for host-only tests. sca_attn_plan gives the same result for the current
+ * device's SM count. Honours sca_set_split_override. Any output may be NULL. */
+SCA_API int sca_attn_plan_for_sms(const sca_metadata* md, int32_t heads, int32_t sms,
+                                  int32_t* n_full, int32_t* n_split, int32_t* chunks,
+                                  uint64_t* workspace_bytes);
+
 /* Process-wide override of the key-split factor used by later attention calls:
  * 0 = automatic (default), 1 = never split, k >= 2 = split every work item
  * after the full waves into k chunks (a test and tuning knob). */

@@ -918,6 +918,19 @@ int sca_attn_plan(const sca_metadata* md, int32_t heads, int32_t* n_full, int32_
   return SCA_OK;
 }
 
+int sca_attn_plan_for_sms(const sca_metadata* md, int32_t heads, int32_t sms, int32_t* n_full,
+                          int32_t* n_split, int32_t* chunks, uint64_t* workspace_bytes) {
+  if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
+  if (heads < 1 || sms < 1) return fail(SCA_ERR_INVALID_ARG, "need heads >= 1 and sms >= 1");
+  int32_t nf, ns, k;
+  choose_plan(md, heads, sms, g_split_override, &nf, &ns, &k);
+  if (n_full) *n_full = nf;
+  if (n_split) *n_split = ns;
+  if (chunks) *chunks = k;
+  if (workspace_bytes) *workspace_bytes = k > 1 ? uint64_t(ns) * uint64_t(k) * kPartialSlotBytes : 0;
+  return SCA_OK;
+}
+
 int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md, int32_t heads,
                                const void* q, const void* k_cur, const void* v_cur, void* o,
                                float* lse, float softmax_scale, void* workspace,

@@ -38,7 +38,8 @@ EXPORTED = (
     "sca_kv_cache_append",
     "sca_kv_cache_truncate", "sca_kv_cache_get", "sca_kv_cache_destroy",
     "sca_action_causal_attn_fwd", "sca_action_causal_attn_fwd_static_ws",
-    "sca_attn_workspace_bytes", "sca_attn_plan", "sca_attn_int8_scratch_bytes",
+    "sca_attn_workspace_bytes", "sca_attn_plan", "sca_attn_plan_for_sms",
+    "sca_attn_int8_scratch_bytes",
     "sca_action_causal_attn_bwd", "sca_attn_bwd_workspace_bytes",
     "sca_set_split_override",
     "sca_last_error", "sca_debug_bounded_wait", "sca_debug_exp2",
@@ -100,6 +101,7 @@ _SIGS = {
                                    _P, ctypes.c_uint64, _P, _P],
     "sca_attn_bwd_workspace_bytes": [_P, _i32, ctypes.POINTER(ctypes.c_uint64)],
     "sca_attn_plan": [_P, _i32, _pi32, _pi32, _pi32],
+    "sca_attn_plan_for_sms": [_P, _i32, _i32, _pi32, _pi32, _pi32, ctypes.POINTER(ctypes.c_uint64)],
     "sca_set_split_override": [_i32],
     "sca_last_error": [],
     "sca_debug_bounded_wait": [_P, _i64, _P],
@@ -420,6 +422,16 @@ def attn_plan(md: Metadata, heads: int) -> dict:
     _check(_lib.sca_attn_plan(md.handle, int(heads), ctypes.byref(a), ctypes.byref(b),
                               ctypes.byref(c)))
     return {"n_full": a.value, "n_split": b.value, "chunks": c.value}
+
+
+def attn_plan_for_sms(md: Metadata, heads: int, sms: int) -> dict:
+    """The work split for a device with ``sms`` SMs (no device needed), with
+    the workspace bytes it takes."""
+    a, b, c = _i32(), _i32(), _i32()
+    w = ctypes.c_uint64()
+    _check(_lib.sca_attn_plan_for_sms(md.handle, int(heads), int(sms), ctypes.byref(a),
+                                      ctypes.byref(b), ctypes.byref(c), ctypes.byref(w)))
+    return {"n_full": a.value, "n_split": b.value, "chunks": c.value, "workspace_bytes": w.value}
 
 
 def set_split_override(chunks: int) -> None:

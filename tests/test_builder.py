@@ -246,3 +246,56 @@ def test_backward_refuses_metadata_not_uploaded():
         sca.action_causal_attn_bwd(md, 2, 16, 16, 16, 16, 16, 16, 16, 16, 16, workspace=256,
                                    workspace_bytes=1 << 20, stream=0)
     assert e.value.code == sca.ERR_INVALID_ARG and "uploaded" in str(e.value)
+
+
+# ---------------------------------------------------------------------------
+# the key-split plan (host-side; sca_attn_plan_for_sms needs no device)
+# ---------------------------------------------------------------------------
+
+SLOT_BYTES = 256 * 128 * 4 + 256 * 8   # one split chunk's fp32 partials: O rows, then (m, l)
+
+
+@pytest.mark.parametrize("make, want", [
+    (W.session_480p_long, (740, 44, 5)),
+    (W.session_480p_single_turn, (740, 44, 4)),
+])
+def test_split_plan_of_the_480p_workloads_on_148_sms(make, want):
+    """The plans the benchmark reported on a 148-SM B200: 49 query-tile pairs
+    x 16 heads = 784 items, five whole waves kept and the 44 left cut into
+    key chunks."""
+    p = make()
+    plan = sca.attn_plan_for_sms(_builder(p), p.heads, 148)
+    assert (plan["n_full"], plan["n_split"], plan["chunks"]) == want
+    assert plan["workspace_bytes"] == want[1] * want[2] * SLOT_BYTES
+
+
+@pytest.mark.parametrize("sms", [1, 7, 132, 148, 160])
+@pytest.mark.parametrize("p", [W.small_session(), W.small_packed(seed=21, n_segments=14),
+                               W.session_480p_single_turn()], ids=lambda p: p.name)
+def test_split_plan_properties(p, sms):
+    md = _builder(p)
+    n_items = (md.counts()["n_q_tiles"] + 1) // 2 * p.heads
+    plan = sca.attn_plan_for_sms(md, p.heads, sms)
+    assert plan["n_full"] + plan["n_split"] == n_items
+    if plan["chunks"] == 1:
+        assert plan["n_split"] == 0 and plan["workspace_bytes"] == 0
+    else:
+        assert plan["chunks"] in (2, 3, 4, 5, 6, 8)
+        assert plan["n_full"] % sms == 0 and plan["n_split"] > 0
+        assert plan["workspace_bytes"] == plan["n_split"] * plan["chunks"] * SLOT_BYTES
+
+
+def test_split_plan_follows_the_override():
+    p = W.session_480p_long()
+    md = _builder(p)
+    try:
+        sca.set_split_override(1)
+        plan = sca.attn_plan_for_sms(md, p.heads, 148)
+        assert (plan["n_full"], plan["n_split"], plan["chunks"]) == (784, 0, 1)
+        sca.set_split_override(3)        # keep all but the last whole wave, cut the rest in 3
+        plan = sca.attn_plan_for_sms(md, p.heads, 148)
+        assert (plan["n_full"], plan["n_split"], plan["chunks"]) == (4 * 148, 784 - 4 * 148, 3)
+    finally:
+        sca.set_split_override(0)
+    with pytest.raises(sca.ScaError):
+        sca.attn_plan_for_sms(md, p.heads, 0)
