@@ -299,3 +299,40 @@ def test_split_plan_follows_the_override():
         sca.set_split_override(0)
     with pytest.raises(sca.ScaError):
         sca.attn_plan_for_sms(md, p.heads, 0)
+
+
+def test_cache_calls_refuse_before_any_gpu_work():
+    """Every refusal of create / append / truncate happens on the host before
+    anything is enqueued, and leaves the cache as it was (fake, aligned
+    device addresses: nothing is dereferenced or launched)."""
+    base = 1 << 20
+    with pytest.raises(sca.ScaError) as e:
+        sca.KVCache(2, 64, base, base + 8, base)
+    assert e.value.code == sca.ERR_MISALIGNED
+    with pytest.raises(sca.ScaError) as e:
+        sca.KVCache(0, 64, base, base, base)
+    assert e.value.code == sca.ERR_INVALID_ARG
+    with pytest.raises(sca.ScaError) as e:
+        sca.KVCache(2, 64, 0, base, base)
+    assert e.value.code == sca.ERR_INVALID_ARG
+
+    cache = sca.KVCache(2, 64, base, base, base)
+    seg = W.Segment(2, 20, 8, (W.Action(4, 0, 1), W.Action(3, 1, 2)))   # 55 tokens
+    big = W.Segment(3, 20, 8)                                           # 68 tokens
+    cases = [
+        (big, base, base, sca.ERR_CAPACITY, "does not fit"),
+        (seg, base + 4, base, sca.ERR_MISALIGNED, "aligned"),
+        (seg, 0, base, sca.ERR_INVALID_ARG, "null k"),
+        (W.Segment(0, 20, 8), base, base, sca.ERR_INVALID_ARG, "num_frames"),
+        (W.Segment(2, 20, 8, (W.Action(4, 1, 3),)), base, base, sca.ERR_INVALID_ARG, "[1, 3)"),
+    ]
+    for s, k, v, code, text in cases:
+        with pytest.raises(sca.ScaError) as e:
+            cache.append(s, k, v, stream=0)
+        assert e.value.code == code and text in str(e.value), (code, str(e.value))
+        assert cache.get() == (0, 0)
+    with pytest.raises(sca.ScaError) as e:
+        cache.truncate(1)
+    assert e.value.code == sca.ERR_INVALID_ARG and cache.get() == (0, 0)
+    cache.truncate(0)
+    assert cache.get() == (0, 0)
