@@ -586,7 +586,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="480p-long-session")
     ap.add_argument("--oracle-rows", type=int, default=384,
                     help="query rows per step of the reference arm")
-    ap.add_argument("--baseline-rows", type=int, default=6144,
+    ap.add_argument("--baseline-rows", type=int, default=8192,
                     help="query rows of the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
