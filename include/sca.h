@@ -33,6 +33,10 @@
  *     [heads][capacity][128] contiguous.
  *   - Every device pointer must be 16-byte aligned (TMA and 16-byte vector
  *     access); otherwise SCA_ERR_MISALIGNED.
+ *   - Threads: different handles may be used from different host threads at
+ *     once. One handle (a metadata or a cache) must not be used by two
+ *     threads at the same time, even through calls that take it as const
+ *     (the attention call caches its work split in the metadata handle).
  */
 #ifndef SCA_H_
 #define SCA_H_

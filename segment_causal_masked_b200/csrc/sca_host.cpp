@@ -16,6 +16,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <numeric>
 #include <queue>
 
@@ -791,7 +792,7 @@ static int make_scale_map(CUtensorMap* m, const float* base, uint64_t rows, uint
 // work split across the SMs
 // ---------------------------------------------------------------------------
 
-static int g_split_override = 0;
+static std::atomic<int> g_split_override{0};  // set by sca_set_split_override, read by planners
 
 static int device_sms(int dev) {
   static int cached[64] = {0};
@@ -866,18 +867,19 @@ static void choose_plan(const sca_metadata* md, int heads, int sms, int forced,
 
 static void plan_for(const sca_metadata* md, int heads, int dev) {
   const int sms = device_sms(dev);
-  if (md->plan_key[0] == heads && md->plan_key[1] == sms && md->plan_key[2] == g_split_override &&
+  const int forced = g_split_override.load();
+  if (md->plan_key[0] == heads && md->plan_key[1] == sms && md->plan_key[2] == forced &&
       md->plan_key[3] == dev)
     return;
   int32_t nf, ns, k;
-  choose_plan(md, heads, sms, g_split_override, &nf, &ns, &k);
+  choose_plan(md, heads, sms, forced, &nf, &ns, &k);
   md->plan_full = nf;
   md->plan_split = ns;
   md->plan_chunks = k;
   md->plan_ws = k > 1 ? uint64_t(ns) * uint64_t(k) * kPartialSlotBytes : 0;
   md->plan_key[0] = heads;
   md->plan_key[1] = sms;
-  md->plan_key[2] = g_split_override;
+  md->plan_key[2] = forced;
   md->plan_key[3] = dev;
 }
 
@@ -923,7 +925,7 @@ int sca_attn_plan_for_sms(const sca_metadata* md, int32_t heads, int32_t sms, in
   if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
   if (heads < 1 || sms < 1) return fail(SCA_ERR_INVALID_ARG, "need heads >= 1 and sms >= 1");
   int32_t nf, ns, k;
-  choose_plan(md, heads, sms, g_split_override, &nf, &ns, &k);
+  choose_plan(md, heads, sms, g_split_override.load(), &nf, &ns, &k);
   if (n_full) *n_full = nf;
   if (n_split) *n_split = ns;
   if (chunks) *chunks = k;
