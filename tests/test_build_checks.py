@@ -101,3 +101,31 @@ def test_plain_c_caller_of_the_abi(tmp_path):
         code, message = lines[key].split(" ", 1)
         assert int(code) == sca.ERR_INVALID_ARG and message, key
     assert "num_frames" in lines["bad_segment"] and "[24, 32)" in lines["bad_window"]
+
+
+def test_binding_constants_match_the_header():
+    """The Python binding restates some of sca.h's constants; read them back
+    from the header so the two cannot drift apart."""
+    import re
+
+    from segment_causal_masked_b200 import sca
+
+    text = open(os.path.join(B.INCLUDE, "sca.h")).read()
+    enums = {m.group(1): int(m.group(2)) for m in re.finditer(r"\b(SCA_\w+)\s*=\s*(-?\d+)", text)}
+    defines = {m.group(1): m.group(2) for m in re.finditer(r"#define\s+(SCA_\w+)\s+(.+)", text)}
+    pairs = {
+        "SCA_OK": sca.OK, "SCA_ERR_INVALID_ARG": sca.ERR_INVALID_ARG,
+        "SCA_ERR_UNSUPPORTED": sca.ERR_UNSUPPORTED, "SCA_ERR_MISALIGNED": sca.ERR_MISALIGNED,
+        "SCA_ERR_CAPACITY": sca.ERR_CAPACITY, "SCA_ERR_CUDA": sca.ERR_CUDA,
+        "SCA_ERR_DEVICE_TIMEOUT": sca.ERR_DEVICE_TIMEOUT, "SCA_ERR_MISMATCH": sca.ERR_MISMATCH,
+        "SCA_TEXTQ_OWN_TAIL": sca.TEXTQ_OWN_TAIL, "SCA_TEXTQ_FULL_SEGMENT": sca.TEXTQ_FULL_SEGMENT,
+        "SCA_TILE_EMPTY": sca.TILE_EMPTY, "SCA_TILE_PARTIAL": sca.TILE_PARTIAL,
+        "SCA_TILE_FULL": sca.TILE_FULL,
+    }
+    for name, value in pairs.items():
+        assert enums[name] == value, name
+    assert int(defines["SCA_HEAD_DIM"]) == sca.HEAD_DIM
+    assert int(defines["SCA_TILE"]) == sca.TILE
+    assert int(defines["SCA_MAX_ACTIONS"]) == sca.MAX_ACTIONS
+    m = re.match(r"\((\d+)ull\s*<<\s*(\d+)\)", defines["SCA_STATIC_WORKSPACE_BYTES"].strip())
+    assert m and int(m.group(1)) << int(m.group(2)) == sca.STATIC_WORKSPACE_BYTES
