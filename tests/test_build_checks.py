@@ -129,3 +129,22 @@ def test_binding_constants_match_the_header():
     assert int(defines["SCA_MAX_ACTIONS"]) == sca.MAX_ACTIONS
     m = re.match(r"\((\d+)ull\s*<<\s*(\d+)\)", defines["SCA_STATIC_WORKSPACE_BYTES"].strip())
     assert m and int(m.group(1)) << int(m.group(2)) == sca.STATIC_WORKSPACE_BYTES
+
+
+def test_binding_signatures_match_the_header_prototypes():
+    """Every exported prototype in sca.h has a ctypes signature in the binding
+    with the same number of arguments."""
+    import re
+
+    from segment_causal_masked_b200 import sca
+
+    text = open(os.path.join(B.INCLUDE, "sca.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    protos = {m.group(1): m.group(2) for m in
+              re.finditer(r"SCA_API\s+[\w\s\*]+?\b(sca_\w+)\s*\(([^)]*)\)\s*;", text, flags=re.S)}
+    assert len(protos) >= 25
+    for name, args in protos.items():
+        n = 0 if args.strip() in ("", "void") else args.count(",") + 1
+        assert name in sca._SIGS, name
+        assert len(sca._SIGS[name]) == n, (name, n, len(sca._SIGS[name]))
+    assert set(protos) == set(sca.EXPORTED)
