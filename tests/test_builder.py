@@ -336,3 +336,17 @@ def test_cache_calls_refuse_before_any_gpu_work():
     assert e.value.code == sca.ERR_INVALID_ARG and cache.get() == (0, 0)
     cache.truncate(0)
     assert cache.get() == (0, 0)
+
+
+def test_unbuilt_or_null_metadata_is_refused_by_every_accessor():
+    md = sca.Metadata()
+    calls = [md.counts, md.schedule, md.descriptors, md.bwd_schedule,
+             lambda: sca.attn_workspace_bytes(md, 2), lambda: sca.attn_int8_scratch_bytes(md, 2),
+             lambda: sca.attn_bwd_workspace_bytes(md, 2), lambda: sca.attn_plan_for_sms(md, 2, 148)]
+    for call in calls:
+        with pytest.raises(sca.ScaError) as e:
+            call()
+        assert e.value.code == sca.ERR_INVALID_ARG and "not built" in str(e.value)
+    assert sca._lib.sca_metadata_get_counts(None, *([None] * 8)) == sca.ERR_INVALID_ARG
+    sca._lib.sca_metadata_destroy(None)      # a no-op
+    sca._lib.sca_kv_cache_destroy(None)
