@@ -65,6 +65,16 @@ WORKLOADS["packed-360k-bwd"] = lambda: dataclasses.replace(W.packed_360k(), name
 WORKLOADS["packed-64k-bwd"] = lambda: dataclasses.replace(W.packed_360k(budget=64_000),
                                                           name="packed-64k-bwd")
 BWD_WORKLOADS = {"packed-360k-bwd", "packed-64k-bwd"}
+# one denoising step of a 480p segment as the distilled model runs it: the
+# metadata built and uploaded once, four attention calls (one per NFE, each
+# with that NFE's own current-segment Q, K and V, seed + nfe) against the same
+# cache, then the append of the segment's K/V (the last NFE's)
+WORKLOADS["480p-single-turn-4nfe"] = lambda: dataclasses.replace(
+    W.session_480p_single_turn(), name="480p-single-turn-4nfe")
+NFE_WORKLOADS = {"480p-single-turn-4nfe": 4}
+# a timed call this long runs at the power-capped clock: its fraction is taken
+# against the sustained bf16 peak, shorter calls against the burst peak
+SUSTAINED_CALL_MS = 500.0
 BWD_FLOP_FACTOR = 2.5   # five products per visible pair against the forward's two
 KERNEL_SOURCES = ["segment_causal_masked_b200/csrc/sca_kernels.cu",
                   "segment_causal_masked_b200/csrc/sca_ptx.cuh",
@@ -220,6 +230,18 @@ class OracleSample:
         return time.perf_counter() - t0
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (first 'model name' of /proc/cpuinfo)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_threads() -> int:
     try:
         import numpy as np  # noqa: F401
@@ -254,7 +276,7 @@ def run_reference(args, problem):
                        "keys": problem.n_key_tokens, "heads": problem.heads,
                        "head_dim": W.HEAD_DIM, "sample_rows_per_step": rows_per_step},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(),
-                             "kind": "oracle", "sample": desc},
+                             "cpu_model": cpu_model(), "kind": "oracle", "sample": desc},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -287,7 +309,8 @@ class Session:
     """One replica of the workload on the current device: a cache holding the
     prior segments, the current segment's Q/K/V, outputs and metadata."""
 
-    def __init__(self, problem, seed: int, int8: bool = False, int8_copy: bool = False):
+    def __init__(self, problem, seed: int, int8: bool = False, int8_copy: bool = False,
+                 nfe: int = 1):
         import torch
 
         from segment_causal_masked_b200 import sca
@@ -321,10 +344,13 @@ class Session:
         # one current segment = an inference step (append after attention);
         # several = a packed training-shaped forward (no cache append)
         self.appends = len(problem.current) == 1
-        self.q = torch.randn(nq, h, 128, generator=g, device=dev).to(bf)
-        self.k_cur = torch.randn(nq, h, 128, generator=g, device=dev).to(bf)
-        self.v_cur = torch.randn(nq, h, 128, generator=g, device=dev).to(bf)
-        self.o = torch.empty(nq, h, 128, dtype=bf, device=dev)
+        # one (Q, K, V) of the current segment per NFE, each drawn afresh
+        self.nfe = nfe
+        self.qkv = [[torch.randn(nq, h, 128, generator=g, device=dev).to(bf) for _ in range(3)]
+                    for _ in range(nfe)]
+        self.q, self.k_cur, self.v_cur = self.qkv[0]
+        self.outs = [torch.empty(nq, h, 128, dtype=bf, device=dev) for _ in range(nfe)]
+        self.o = self.outs[0]
         self.lse = torch.empty(h, nq, dtype=torch.float32, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.md = sca.build_for(problem)
@@ -374,25 +400,28 @@ class Session:
         if ev is not None:
             ev[1].record(self.stream)
 
-    def step(self, q=None, k_cur=None, v_cur=None, o=None, ev=None):
-        """One pass of the hot path; `ev` = (start, end) events around the
-        attention kernel."""
+    def step(self, ins=None, outs=None, ev=None):
+        """One pass of the hot path: the metadata built and uploaded, one
+        attention call per NFE, then the append. ``ins`` = [q, k_cur, v_cur]
+        per NFE and ``outs`` = [o] per NFE (the session's own by default);
+        ``ev`` = one (start, end) event pair per attention call."""
         sca, p = self.sca, self.p
         s = self.stream.cuda_stream
         sca.build_for(p, self.md)
         self.md.upload(s)
-        if ev is not None:
-            ev[0].record(self.stream)
-        sca.action_causal_attn_fwd(self.cache, self.md, p.heads, self.q if q is None else q,
-                                   self.k_cur if k_cur is None else k_cur,
-                                   self.v_cur if v_cur is None else v_cur,
-                                   self.o if o is None else o, self.lse, p.softmax_scale,
-                                   self.workspace, None, self.status, s)
-        if ev is not None:
-            ev[1].record(self.stream)
+        qkv = self.qkv if ins is None else [ins[3 * i:3 * i + 3] for i in range(self.nfe)]
+        outs = self.outs if outs is None else outs
+        for i in range(self.nfe):
+            q, k_cur, v_cur = qkv[i]
+            if ev is not None:
+                ev[i][0].record(self.stream)
+            sca.action_causal_attn_fwd(self.cache, self.md, p.heads, q, k_cur, v_cur, outs[i],
+                                       self.lse, p.softmax_scale, self.workspace, None,
+                                       self.status, s)
+            if ev is not None:
+                ev[i][1].record(self.stream)
         if self.appends:  # inference: the generated segment joins the cache
-            self.cache.append(p.current[0], self.k_cur if k_cur is None else k_cur,
-                              self.v_cur if v_cur is None else v_cur, s)
+            self.cache.append(p.current[0], qkv[-1][1], qkv[-1][2], s)
             self.cache.truncate(self.n_prior)
 
 
@@ -421,24 +450,28 @@ def run_native(args, problem):
     int8 = args.workload in INT8_WORKLOADS
     bwd = args.workload in BWD_WORKLOADS
     int8_copy = args.workload in INT8_COPY_WORKLOADS
-    sess = Session(problem, seed=1000 * 2 + rank, int8=int8, int8_copy=int8_copy)
+    nfe = NFE_WORKLOADS.get(args.workload, 1)
+    sess = Session(problem, seed=1000 * 2 + rank, int8=int8, int8_copy=int8_copy, nfe=nfe)
     from segment_causal_masked_b200 import sca
     sca_md = sca.build_for(problem)
     counts = sca_md.counts()
     A = counts["unmasked_pairs"]
-    flops = effective_flops(problem, A)
+    flops_call = effective_flops(problem, A)   # one attention call (one NFE)
+    flops = nfe * flops_call                     # one step
     step = sess.step
     if bwd:
         sess.prepare_backward(1000 * 3 + rank)
         flops *= BWD_FLOP_FACTOR
+        flops_call = flops
         step = sess.step_backward
 
     # ---- device-resident timing
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+    # one (start, end) pair around every attention call (the backward: the call)
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(1 if bwd else nfe)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     barrier()
@@ -446,7 +479,7 @@ def run_native(args, problem):
     clocks.start()
     t_start.record(sess.stream)
     for i in range(args.steps):
-        step(ev=evs[i])
+        step(ev=evs[i][0] if bwd else evs[i])
     t_end.record(sess.stream)
     torch.cuda.synchronize()
     clock_info = clocks.stop()
@@ -454,7 +487,7 @@ def run_native(args, problem):
     if int(sess.status.item()) != 0:
         raise SystemExit(f"device status {int(sess.status.item())}")
     ms_total = max_over_ranks(t_start.elapsed_time(t_end))
-    attn_ms = [a.elapsed_time(b) for a, b in evs]
+    attn_ms = [a.elapsed_time(b) for calls in evs for a, b in calls]
     attn_avg = max_over_ranks(statistics.mean(attn_ms))
     ms_step = ms_total / args.steps
     value = whole_job_tflops(world, flops, args.steps, ms_total)
@@ -474,12 +507,12 @@ def run_native(args, problem):
         def run(ins, outs):
             q, k, v, o, lse, d_o = ins
             sess.step_backward(q=q, k=k, v=v, o=o, lse=lse, d_o=d_o, grads=outs)
-    else:     # inputs q, k_cur, v_cur; result o
-        host_in = [t.cpu().pin_memory() for t in (sess.q, sess.k_cur, sess.v_cur)]
-        host_out = [torch.empty(nq, h, 128, **pin)]
+    else:     # inputs q, k_cur, v_cur of every NFE; result o of every NFE
+        host_in = [t.cpu().pin_memory() for qkv in sess.qkv for t in qkv]
+        host_out = [torch.empty(nq, h, 128, **pin) for _ in range(nfe)]
 
         def run(ins, outs):
-            sess.step(q=ins[0], k_cur=ins[1], v_cur=ins[2], o=outs[0])
+            sess.step(ins=ins, outs=outs)
     dev_in = [[torch.empty_like(t, device="cuda") for t in host_in] for _ in range(2)]
     dev_out = [[torch.empty_like(t, device="cuda") for t in host_out] for _ in range(2)]
     bytes_in = sum(t.numel() * t.element_size() for t in host_in)
@@ -534,8 +567,9 @@ def run_native(args, problem):
 
     if rank == 0:
         peaks = measured_peaks()
-        peak = float(peaks["bf16_tflops"])
-        achieved = flops / (attn_avg * 1e-3) / 1e12
+        sustained = attn_avg >= SUSTAINED_CALL_MS
+        peak = float(peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"])
+        achieved = flops_call / (attn_avg * 1e-3) / 1e12
         traffic = None if bwd else stored_traffic("attn_fwd_kernel", problem.name)
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
@@ -548,10 +582,15 @@ def run_native(args, problem):
                        "effective_flop_per_step": flops,
                        "step": ("attention backward (D and LSE, dQ, dK and dV kernels); the "
                                 "forward that produced O and LSE ran once before timing" if bwd
+                                else ("metadata build+upload, %d attention forwards (one per "
+                                      "NFE, each with its own current-segment Q, K, V), "
+                                      "kv_cache_append" % nfe) if nfe > 1
                                 else "metadata build+upload, attention forward, kv_cache_append"
                                 if sess.appends else "metadata build+upload, attention forward"),
+                       "nfe": nfe,
                        "flop_count": ("10·d·H·A (five products per visible pair)" if bwd
-                                      else "4·d·H·A (two products per visible pair)"),
+                                      else "4·d·H·A (two products per visible pair)"
+                                      + (" per NFE" if nfe > 1 else "")),
                        "kv_cache": ("int8 codes + fp32 row scales" + (", dequantised once per call"
                                     " into a bf16 copy in the workspace" if int8_copy else
                                     ", dequantised tile by tile in the kernel")) if int8 else "bf16",
@@ -564,11 +603,16 @@ def run_native(args, problem):
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                          "kernel": ("bwd_prep_kernel + bwd_dq_kernel + bwd_dkdv_kernel" if bwd
                                     else "attn_fwd_kernel"), "kernel_ms": attn_avg,
-                         "peak_source": f"{peaks['source']} bf16 dense (burst)"},
+                         "kernel_ms_is": ("per backward call" if bwd else
+                                          "per attention call (one NFE)"),
+                         "peak_source": f"{peaks['source']} bf16 dense "
+                                        + ("(sustained: the call lasts over %.1f s)"
+                                           % (SUSTAINED_CALL_MS / 1e3) if sustained
+                                           else "(burst)")},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": bytes_in,
                     "d2h_bytes_per_step": bytes_out, "ms_per_step": e2e_ms / args.steps},
-            "gpu_launches": (3 if bwd else 1 + int(sess.appends) + int(sess.splits)
-                             + int(int8_copy)) * args.steps,
+            "gpu_launches": (3 if bwd else nfe * (1 + int(sess.splits) + int(int8_copy))
+                             + int(sess.appends)) * args.steps,
             "clocks": clock_info,
         }
         if not args.no_cpu_baseline:
@@ -576,8 +620,8 @@ def run_native(args, problem):
                                   backward=bwd)
             dt = sample.run()
             line["cpu_baseline"] = {"value": sample.flops / dt / 1e12, "unit": "TFLOP/s",
-                                    "cores": cpu_threads(), "kind": "oracle",
-                                    "sample": sample.desc, "seconds": dt}
+                                    "cores": cpu_threads(), "cpu_model": cpu_model(),
+                                    "kind": "oracle", "sample": sample.desc, "seconds": dt}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

@@ -310,10 +310,24 @@ SCA_API int sca_attn_plan_for_sms(const sca_metadata* md, int32_t heads, int32_t
                                   int32_t* n_full, int32_t* n_split, int32_t* chunks,
                                   uint64_t* workspace_bytes);
 
-/* Process-wide override of the key-split factor used by later attention calls:
+/* Override of the key-split factor used by later attention calls made from
+ * the calling host thread (other threads keep their own setting, so a test
+ * or tuning loop on one thread cannot change another thread's calls):
  * 0 = automatic (default), 1 = never split, k >= 2 = split every work item
  * after the full waves into k chunks (a test and tuning knob). */
 SCA_API int sca_set_split_override(int32_t chunks);
+
+/* Limit, in nanoseconds, of every pipeline wait inside the kernels (for a
+ * tile load, a product or a handshake between warps) of later attention calls
+ * made from the calling host thread: [0, 10 s], default 2 s. A wait that runs
+ * out stores SCA_ERR_DEVICE_TIMEOUT in the call's device status word and makes
+ * every CTA of the kernel stop issuing work; the output is then undefined.
+ * Before a CTA frees its tensor memory and exits, it still waits for the
+ * loads and products it has already issued, with a fixed limit of its own
+ * (2 s) that this setting does not change, so the device stays usable. A test
+ * and debugging knob: 0 makes a call give up at its first wait that is not
+ * complete at once, which exercises that abort path on the real kernels. */
+SCA_API int sca_set_pipeline_timeout_ns(int64_t ns);
 
 /* Attention forward for callers that cannot allocate device memory (no
  * counterpart in the Hy-Nomas pages; a deployment convenience). Some callers
@@ -326,16 +340,25 @@ SCA_API int sca_set_split_override(int32_t chunks);
  * SCA_STATIC_WORKSPACE_BYTES that is part of the library; it allocates
  * nothing. Arguments and results are those of sca_action_causal_attn_fwd,
  * without the workspace.
- *   - Limit: if the call's split plan needs more scratch than the array holds
- *     (sca_attn_workspace_bytes), it returns SCA_ERR_CAPACITY and launches
- *     nothing.
+ *   - Limit: the array holds 32 MiB, enough for the automatic split plans
+ *     of the 480p single-turn and long-session layouts (16 heads; with or
+ *     without a sliding window or a quarter of the video blocks) on a
+ *     148-SM B200. If the automatic plan needs more (sca_attn_workspace_bytes;
+ *     other layouts, other SM counts), the call runs every work item whole,
+ *     which needs no scratch. If a split forced with sca_set_split_override
+ *     needs more, it returns SCA_ERR_CAPACITY and launches nothing.
+ *   - INT8 cache: when the split partials plus a bf16 copy of the cached K
+ *     and V (sca_attn_int8_scratch_bytes) fit in the array, the call also
+ *     dequantises the cache once into the array and runs the bf16 kernel on
+ *     the copy, exactly as sca_action_causal_attn_fwd does with a workspace
+ *     that large; otherwise it dequantises tile by tile. Same result.
  *   - Set-up: the first call on each device (with that device current) looks
- *     up the array's device address once; make that first call before any
- *     stream capture.
+ *     up the array's device address, once per context (again after a
+ *     cudaDeviceReset); make that first call before any stream capture.
  *   - Sharing: every call, on every stream, uses the same array, which keeps
  *     the last call's contents. Nothing in it needs to start at zero (a call
- *     reads only partials it wrote itself), but calls that overlap on the GPU
- *     race: order them (one stream, or events).
+ *     reads only partials and copies it wrote itself), but calls that
+ *     overlap on the GPU race: order them (one stream, or events).
  *   - Memory: every GPU that loads the library holds the array until the
  *     process exits. */
 #define SCA_STATIC_WORKSPACE_BYTES (32ull << 20)
@@ -392,6 +415,15 @@ SCA_API int sca_attn_bwd_workspace_bytes(const sca_metadata* md, int32_t heads, 
 /* Message of the calling thread's last failure ("" if none). */
 SCA_API const char* sca_last_error(void);
 
+/* Read a device status word (the dev_status of the attention calls): waits
+ * for the work queued on `stream` so far, copies the word to the host and
+ * returns it: SCA_OK when no kernel reported a failure, else the negative
+ * code a kernel stored (SCA_ERR_DEVICE_TIMEOUT, SCA_ERR_MISALIGNED), with a
+ * message from sca_last_error. SCA_ERR_CUDA if the copy itself fails,
+ * SCA_ERR_INVALID_ARG for a null pointer. The word is left as it is; the
+ * caller clears it (a 4-byte memset) before reusing it. */
+SCA_API int sca_read_device_status(const int32_t* dev_status, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Self-test of the device-side bounded wait: one block waits on an mbarrier
  * that nothing completes, gives up after `timeout_ns` nanoseconds, writes
@@ -400,11 +432,6 @@ SCA_API const char* sca_last_error(void);
  * ------------------------------------------------------------------------- */
 SCA_API int sca_debug_bounded_wait(int32_t* dev_status, int64_t timeout_ns, void* stream);
 
-/* Evaluate, for n floats x (device, x <= 8), the two exponentials the
- * attention kernel uses: y_poly = 2^x by range reduction and a fitted cubic
- * on the FMA pipe, y_mufu = 2^x by the ex2.approx instruction. For testing
- * the first against the second and against float64. */
-SCA_API int sca_debug_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n, void* stream);
 
 #ifdef __cplusplus
 }

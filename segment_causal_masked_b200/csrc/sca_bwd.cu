@@ -29,6 +29,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "sca_internal.h"
 #include "sca_ptx.cuh"
 
@@ -290,7 +292,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
         ok = wait_bar(bar(kQBarVE + vs), (uint32_t(j / kQVSlots) & 1u) ^ 1u, ctl, p.status,
                       p.timeout_ns);
         if (!ok) {
-          wait_bounded(bar(kQBarKF + ks), uint32_t(j / kQKSlots) & 1u, ctl, nullptr, p.timeout_ns);
+          wait_drain(bar(kQBarKF + ks), uint32_t(j / kQKSlots) & 1u);  // this K load is armed
           break;
         }
         mbar_expect_tx(bar(kQBarVF + vs), kBTile);
@@ -298,17 +300,15 @@ __global__ void __launch_bounds__(kBThreads, 1)
         tma_load_3d(sbase + kQOffV + vs * kBTile + kBHalf, &tm_v, bar(kQBarVF + vs), 64, head, row);
         ++j;
       }
-      if (!ok) {
-        // drain: every armed load lands before the CTA can exit (the latest
-        // load of each slot is among the last kQKSlots / kQVSlots)
-        for (int i = j - kQKSlots < 0 ? 0 : j - kQKSlots; i < j; ++i)
-          wait_bounded(bar(kQBarKF + i % kQKSlots), uint32_t(i / kQKSlots) & 1u, ctl, nullptr,
-                       p.timeout_ns);
-        for (int i = j - kQVSlots < 0 ? 0 : j - kQVSlots; i < j; ++i)
-          wait_bounded(bar(kQBarVF + i % kQVSlots), uint32_t(i / kQVSlots) & 1u, ctl, nullptr,
-                       p.timeout_ns);
-        wait_bounded(bar(kQBarQD), 0, ctl, nullptr, p.timeout_ns);
-      }
+      // Drain, also after a normal end (where it finds every load landed):
+      // every armed load lands before the CTA can exit, even when a consumer
+      // gave up (the latest load of each slot is among the last kQKSlots /
+      // kQVSlots)
+      for (int i = j - kQKSlots < 0 ? 0 : j - kQKSlots; i < j; ++i)
+        wait_drain(bar(kQBarKF + i % kQKSlots), uint32_t(i / kQKSlots) & 1u);
+      for (int i = j - kQVSlots < 0 ? 0 : j - kQVSlots; i < j; ++i)
+        wait_drain(bar(kQBarVF + i % kQVSlots), uint32_t(i / kQVSlots) & 1u);
+      wait_drain(bar(kQBarQD), 0);
     } else if (warp == 9) {
       // ---------------------------------------------------------------- MMA
       int n = 0;  // live key tiles of this query tile, counted by the warp
@@ -378,7 +378,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
         mma_commit(bar(kQBarDone));
         mma_commit(bar(kQBarDrain));
-        wait_bounded(bar(kQBarDrain), 0, ctl, nullptr, p.timeout_ns);
+        wait_drain(bar(kQBarDrain), 0);
       }
       __syncwarp();
     }
@@ -402,10 +402,13 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const int c0 = 64 * half;
     bool ok = true;
     int j = 0;
+    uint32_t e_next = len > 0 ? list[0] : 0u;
     for (int e = 0; e < len; ++e) {
-      const uint32_t cls = cls_of(e);
+      const uint32_t entry = e_next;
+      if (e + 1 < len) e_next = list[e + 1];   // prefetch the next schedule entry
+      const uint32_t cls = (entry >> (24 + 2 * t)) & 3u;
       if (cls == SCA_TILE_EMPTY) continue;
-      const int tile = int(list[e] & kPairTileMask);
+      const int tile = int(entry & kPairTileMask);
       uint32_t vis[2] = {0u, 0u};
       if (cls == SCA_TILE_PARTIAL) {
         for (int i = p.run_ptr[tile]; i < p.run_ptr[tile + 1]; ++i) {
@@ -559,11 +562,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
       tma_load_3d(sbase + kKOffV, &tm_v, bar(kKBarKV), 0, head, k0);
       tma_load_3d(sbase + kKOffV + kBHalf, &tm_v, bar(kKBarKV), 64, head, k0);
       int i = 0;
-      bool ok = true;
       for (; i < n; ++i) {
         const int s = i % kKStages;
-        if (!(ok = wait_bar(bar(kKBarE + s), (uint32_t(i / kKStages) & 1u) ^ 1u, ctl, p.status,
-                            p.timeout_ns)))
+        if (!wait_bar(bar(kKBarE + s), (uint32_t(i / kKStages) & 1u) ^ 1u, ctl, p.status,
+                      p.timeout_ns))
           break;
         const int q0 = int(list[i] & kPairTileMask) * 128;
         const uint32_t st = sbase + stage(i), fb = bar(kKBarF + s);
@@ -575,12 +577,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
         tma_load_2d(st + 2 * kBTile, &tm_dl, fb, q0, head);
         tma_load_2d(st + 2 * kBTile + 512, &tm_dl, fb, q0, p.heads + head);
       }
-      if (!ok) {
-        for (int i2 = i - kKStages < 0 ? 0 : i - kKStages; i2 < i; ++i2)
-          wait_bounded(bar(kKBarF + i2 % kKStages), uint32_t(i2 / kKStages) & 1u, ctl, nullptr,
-                       p.timeout_ns);
-        wait_bounded(bar(kKBarKV), 0, ctl, nullptr, p.timeout_ns);
-      }
+      // Drain, also after a normal end: every armed load lands before the
+      // CTA can exit, even when a consumer gave up.
+      for (int i2 = i - kKStages < 0 ? 0 : i - kKStages; i2 < i; ++i2)
+        wait_drain(bar(kKBarF + i2 % kKStages), uint32_t(i2 / kKStages) & 1u);
+      wait_drain(bar(kKBarKV), 0);
     } else if (warp == 9 && lane == 0) {
       // ---------------------------------------------------------------- MMA
       const uint64_t dK = desc_kmajor(sbase + kKOffK), dV = desc_kmajor(sbase + kKOffV);
@@ -624,7 +625,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
       }
       mma_commit(bar(kKBarDone));
       mma_commit(bar(kKBarDrain));
-      wait_bounded(bar(kKBarDrain), 0, ctl, nullptr, p.timeout_ns);
+      wait_drain(bar(kKBarDrain), 0);
     }
     __syncwarp();
   } else {
@@ -639,8 +640,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const uint64_t c2 = f2(p.scale_log2, p.scale_log2);
     bool ok = true;
     int i = 0;
+    uint32_t e_next = n > 0 ? list[0] : 0u;
     for (; i < n; ++i) {
-      const uint32_t e = list[i];
+      const uint32_t e = e_next;
+      if (i + 1 < n) e_next = list[i + 1];     // prefetch the next schedule entry
       const int qt = int(e & kPairTileMask);
       const uint32_t cls = e >> 24;
       uint32_t vis[2] = {0u, 0u};  // query blocks b = 0, 1
@@ -679,15 +682,19 @@ __global__ void __launch_bounds__(kBThreads, 1)
       // per query column -D and -L as pairs; block b covers queries
       // [64 b + 32 half, +32). Pᵀ goes to Sᵀ columns [32 half + 16 b, +16),
       // dSᵀ to [64 + 32 half + 16 b, +16): only columns this thread has read.
-      const uint64_t* ndl = reinterpret_cast<const uint64_t*>(smem + stage(i) + 2 * kBTile);
+      // (16-byte broadcast loads: four columns' -D or -L per load)
+      const ulonglong2* ndl = reinterpret_cast<const ulonglong2*>(smem + stage(i) + 2 * kBTile);
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         const int cb = 64 * b + 32 * half;
         uint64_t nd2[16], nl2[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          nd2[k] = ndl[cb / 2 + k];
-          nl2[k] = ndl[64 + cb / 2 + k];
+        for (int k = 0; k < 8; ++k) {
+          const ulonglong2 d = ndl[cb / 4 + k], l = ndl[32 + cb / 4 + k];
+          nd2[2 * k] = d.x;
+          nd2[2 * k + 1] = d.y;
+          nl2[2 * k] = l.x;
+          nl2[2 * k + 1] = l.y;
         }
         const float(&sb)[32] = *reinterpret_cast<const float(*)[32]>(s + 32 * b);
         const float(&dpb)[32] = *reinterpret_cast<const float(*)[32]>(dp + 32 * b);
@@ -741,17 +748,19 @@ __global__ void __launch_bounds__(kBThreads, 1)
 }
 
 cudaError_t launch_backward(const BwdMaps& maps, const BwdArgs& args, cudaStream_t stream) {
-  static int configured_mask = 0;
+  // devices whose kernel attributes are set (a set bit; set at most once
+  // per device, safely from several host threads)
+  static std::atomic<uint32_t> configured_mask{0u};
   int dev = 0, sms = 148;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 31 || !(configured_mask & (1 << dev))) {
+  if (dev >= 31 || !(configured_mask.load() & (1u << dev))) {
     e = cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kQSmem));
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                int(kKSmem));
     if (e != cudaSuccess) return e;
-    if (dev < 31) configured_mask |= 1 << dev;
+    if (dev < 31) configured_mask.fetch_or(1u << dev);
   }
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t rows = int64_t(args.n_pad) * args.heads;

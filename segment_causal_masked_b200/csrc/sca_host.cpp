@@ -151,6 +151,17 @@ uint8_t classify(const TileSummary& q, const TileSummary& k, uint32_t window) {
 
 }  // namespace
 
+// Set by sca_set_split_override and read by the planners of the same host
+// thread only, so a test or tuning loop on one thread cannot change the plan
+// of a call another thread is making.
+static thread_local int g_split_override = 0;
+
+int split_override() { return g_split_override; }
+
+// Limit of the kernels' pipeline waits for calls from this host thread
+// (sca_set_pipeline_timeout_ns).
+static thread_local unsigned long long g_pipeline_timeout_ns = 2000000000ull;
+
 }  // namespace sca
 
 using namespace sca;
@@ -723,17 +734,17 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// Looked up once (a function-local static is initialised exactly once, also
+// when several host threads get here at the same time).
 static EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+      return reinterpret_cast<EncodeTiledFn>(p);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -792,14 +803,16 @@ static int make_scale_map(CUtensorMap* m, const float* base, uint64_t rows, uint
 // work split across the SMs
 // ---------------------------------------------------------------------------
 
-static std::atomic<int> g_split_override{0};  // set by sca_set_split_override, read by planners
 
 static int device_sms(int dev) {
-  static int cached[64] = {0};
-  if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev];
+  static std::atomic<int> cached[64] = {};
+  if (dev >= 0 && dev < 64) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c) return c;
+  }
   int sms = 148;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 148;
-  if (dev >= 0 && dev < 64) cached[dev] = sms;
+  if (dev >= 0 && dev < 64) cached[dev].store(sms, std::memory_order_relaxed);
   return sms;
 }
 
@@ -867,7 +880,7 @@ static void choose_plan(const sca_metadata* md, int heads, int sms, int forced,
 
 static void plan_for(const sca_metadata* md, int heads, int dev) {
   const int sms = device_sms(dev);
-  const int forced = g_split_override.load();
+  const int forced = g_split_override;
   if (md->plan_key[0] == heads && md->plan_key[1] == sms && md->plan_key[2] == forced &&
       md->plan_key[3] == dev)
     return;
@@ -881,6 +894,13 @@ static void plan_for(const sca_metadata* md, int heads, int dev) {
   md->plan_key[1] = sms;
   md->plan_key[2] = forced;
   md->plan_key[3] = dev;
+}
+
+int sca_set_pipeline_timeout_ns(int64_t ns) {
+  if (ns < 0 || ns > 10000000000LL)
+    return fail(SCA_ERR_INVALID_ARG, "pipeline timeout must be in [0, 10 s]");
+  g_pipeline_timeout_ns = (unsigned long long)ns;
+  return SCA_OK;
 }
 
 int sca_set_split_override(int32_t chunks) {
@@ -925,7 +945,7 @@ int sca_attn_plan_for_sms(const sca_metadata* md, int32_t heads, int32_t sms, in
   if (!md || !md->built) return fail(SCA_ERR_INVALID_ARG, "metadata not built");
   if (heads < 1 || sms < 1) return fail(SCA_ERR_INVALID_ARG, "need heads >= 1 and sms >= 1");
   int32_t nf, ns, k;
-  choose_plan(md, heads, sms, g_split_override.load(), &nf, &ns, &k);
+  choose_plan(md, heads, sms, g_split_override, &nf, &ns, &k);
   if (n_full) *n_full = nf;
   if (n_split) *n_split = ns;
   if (chunks) *chunks = k;
@@ -1031,7 +1051,7 @@ int sca_action_causal_attn_fwd(const sca_kv_cache* cache, const sca_metadata* md
   a.n_pairs = md->n_pairs;
   a.history = md->history;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
-  a.timeout_ns = 2000000000ull;
+  a.timeout_ns = g_pipeline_timeout_ns;
   const bool split = md->plan_chunks > 1 && workspace && workspace_bytes >= md->plan_ws;
   a.n_full = split ? md->plan_full : md->n_pairs * heads;
   a.n_split = split ? md->plan_split : 0;
@@ -1126,14 +1146,27 @@ int sca_action_causal_attn_bwd(const sca_metadata* md, int32_t heads, const void
   a.history = md->history;
   a.scale = softmax_scale;
   a.scale_log2 = softmax_scale * 1.4426950408889634f;
-  a.timeout_ns = 2000000000ull;
+  a.timeout_ns = g_pipeline_timeout_ns;
   return check_cuda(launch_backward(maps, a, static_cast<cudaStream_t>(stream)), "backward launch");
 }
 
-int sca_debug_exp2(const float* x, float* y_poly, float* y_mufu, int64_t n, void* stream) {
-  if (!x || !y_poly || !y_mufu || n < 0) return fail(SCA_ERR_INVALID_ARG, "bad exp2 arguments");
-  return check_cuda(launch_exp2_eval(x, y_poly, y_mufu, n, static_cast<cudaStream_t>(stream)),
-                    "exp2 launch");
+int sca_read_device_status(const int32_t* dev_status, void* stream) {
+  if (!dev_status) return fail(SCA_ERR_INVALID_ARG, "null status word");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (int rc = check_cuda(cudaMemcpyAsync(&v, dev_status, sizeof(v), cudaMemcpyDeviceToHost, st),
+                          "cudaMemcpyAsync(status)"))
+    return rc;
+  if (int rc = check_cuda(cudaStreamSynchronize(st), "cudaStreamSynchronize")) return rc;
+  switch (v) {
+    case SCA_OK: return SCA_OK;
+    case SCA_ERR_DEVICE_TIMEOUT:
+      return fail(v, "a kernel's bounded wait ran out (device status %d)", v);
+    case SCA_ERR_MISALIGNED:
+      return fail(v, "a kernel's shared-memory window was misaligned (device status %d)", v);
+    default:
+      return fail(v < 0 ? v : SCA_ERR_CUDA, "device status word holds %d", v);
+  }
 }
 
 int sca_debug_bounded_wait(int32_t* dev_status, int64_t timeout_ns, void* stream) {

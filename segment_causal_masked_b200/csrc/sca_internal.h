@@ -42,6 +42,8 @@ struct SegLayout {
 int fail(int code, const char* fmt, ...);
 int check_cuda(cudaError_t e, const char* what);
 int read_segment(const sca_segment* s, SegLayout* out);
+// The calling thread's key-split override (sca_set_split_override).
+int split_override();
 
 // Descriptor word of token `t` (0-based inside the segment).
 uint32_t key_descriptor(const SegLayout& s, uint32_t seg_index, int64_t t);
@@ -178,8 +180,6 @@ struct BwdMaps {
 cudaError_t launch_backward(const BwdMaps& maps, const BwdArgs& args, cudaStream_t stream);
 cudaError_t launch_bounded_wait(int32_t* status, unsigned long long timeout_ns,
                                 cudaStream_t stream);
-cudaError_t launch_exp2_eval(const float* x, float* y_poly, float* y_mufu, int64_t n,
-                             cudaStream_t stream);
 
 size_t attention_smem_bytes(bool int8_cache);
 

@@ -29,6 +29,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "sca_internal.h"
 #include "sca_ptx.cuh"
 
@@ -205,9 +207,6 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
 // p = exp2(x * scale - m) for one row's 128 scores, summed into `acc` and
 // written as bf16 pairs over the first 64 TMEM columns of the row's S (P
 // chunk c lands in S chunk c/2, whose scores are already in registers).
-// kEvery > 0: every kEvery-th pair of exponentials is evaluated on the FMA
-// pipe (exp2_poly2, finite inputs only) instead of the MUFU.
-template <int kEvery>
 __device__ __forceinline__ void exp_pack_store(const float (&x)[128], uint64_t scale2,
                                                uint64_t negm2, uint32_t tS, uint64_t (&acc)[2]) {
 #pragma unroll
@@ -215,14 +214,9 @@ __device__ __forceinline__ void exp_pack_store(const float (&x)[128], uint64_t s
     uint32_t pk[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      float x0, x1, p0, p1;
+      float x0, x1;
       unf2(fma2(f2(x[32 * c + 2 * i], x[32 * c + 2 * i + 1]), scale2, negm2), x0, x1);
-      if (kEvery > 0 && (i % (kEvery > 0 ? kEvery : 1)) == kEvery - 1) {
-        exp2_poly2(x0, x1, p0, p1);
-      } else {
-        p0 = ex2(x0);
-        p1 = ex2(x1);
-      }
+      const float p0 = ex2(x0), p1 = ex2(x1);
       acc[i & 1] = add2(acc[i & 1], f2(p0, p1));
       pk[i] = pack_bf16(p0, p1);
     }
@@ -302,7 +296,6 @@ constexpr int kMmaWarp = 9;
 constexpr uint32_t kHalf = 128 * 64 * 2;  // one 128-row x 64-column bf16 box: 16 KB
 constexpr uint32_t kTile = 2 * kHalf;     // 128 x 128 bf16: 32 KB
 constexpr float kRescaleThreshold = 8.0f; // log2 units: p stays <= 2^8 between rescales
-constexpr int kPolyEvery = 0;             // every n-th exponential pair of FULL tiles on the FMA pipe (0: none)
 
 // shared-memory map (offsets from a 1024-aligned base)
 constexpr uint32_t kOffQ = 0;                            // Q0, Q1
@@ -513,24 +506,21 @@ __global__ void __launch_bounds__(threads_for(kInt8), 1)
           }
         }
       }
-      if (!ok) {
-        // drain: let every armed load land before the CTA can exit. The
-        // latest load of each ring slot is among the last kRing issued (the
-        // staged loads among them filled no ring slot); that of each code
-        // slot among the last kCodeSlots staged loads, which form a prefix.
-        for (int back = 1; back <= kRing && it - back >= 0; ++back) {
-          const int i2 = it - back;
-          if (!staged(i2))
-            wait_bounded(bar(kBarFull + i2 % kRing), uint32_t(i2 / kRing) & 1u, ctl, nullptr,
-                         p.timeout_ns);
-        }
-        int n_staged = 0;
-        while (n_staged < it && staged(n_staged)) ++n_staged;
-        for (int i2 = n_staged - kCodeSlots < 0 ? 0 : n_staged - kCodeSlots; i2 < n_staged; ++i2)
-          wait_bounded(bar(kBarCodeFull + i2 % kCodeSlots), uint32_t(i2 / kCodeSlots) & 1u, ctl,
-                       nullptr, p.timeout_ns);
-        wait_bounded(bar(kBarQ), 0, ctl, nullptr, p.timeout_ns);
+      // Drain, also after a normal end (where it finds every load landed):
+      // every armed load lands before the CTA can exit, even when a consumer
+      // gave up and will never wait for it. The latest load of each ring
+      // slot is among the last kRing issued (the staged loads among them
+      // filled no ring slot); that of each code slot among the last
+      // kCodeSlots staged loads, which form a prefix.
+      for (int back = 1; back <= kRing && it - back >= 0; ++back) {
+        const int i2 = it - back;
+        if (!staged(i2)) wait_drain(bar(kBarFull + i2 % kRing), uint32_t(i2 / kRing) & 1u);
       }
+      int n_staged = 0;
+      while (n_staged < it && staged(n_staged)) ++n_staged;
+      for (int i2 = n_staged - kCodeSlots < 0 ? 0 : n_staged - kCodeSlots; i2 < n_staged; ++i2)
+        wait_drain(bar(kBarCodeFull + i2 % kCodeSlots), uint32_t(i2 / kCodeSlots) & 1u);
+      wait_drain(bar(kBarQ), 0);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -596,7 +586,7 @@ __global__ void __launch_bounds__(threads_for(kInt8), 1)
       mma_commit(bar(kBarO + 1));
       // every MMA has finished before this thread leaves (also on abort)
       mma_commit(bar(kBarDrain));
-      wait_bounded(bar(kBarDrain), 0, ctl, nullptr, p.timeout_ns);
+      wait_drain(bar(kBarDrain), 0);
     }
     __syncwarp();
   }
@@ -678,14 +668,8 @@ __global__ void __launch_bounds__(threads_for(kInt8), 1)
         const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
         const uint64_t negm2 = f2(neg_m, neg_m);
         uint64_t acc[2] = {0ull, 0ull};  // packed partial sums
-        // p = exp2(s * scale_log2 - m), row sum, bf16 P. FULL tiles (no -inf)
-        // may send part of the exponentials to the FMA pipe; the choice is
-        // made once per tile so the compiler keeps the two paths apart.
-        if (cls == SCA_TILE_FULL) {
-          exp_pack_store<kPolyEvery>(x, scale2, negm2, tS, acc);
-        } else {
-          exp_pack_store<0>(x, scale2, negm2, tS, acc);
-        }
+        // p = exp2(s * scale_log2 - m), row sum, bf16 P
+        exp_pack_store(x, scale2, negm2, tS, acc);
         float a0, a1;
         unf2(add2(acc[0], acc[1]), a0, a1);
         // one explicit rounding (l alpha + sum), so every instantiation of
@@ -781,16 +765,18 @@ __global__ void __launch_bounds__(threads_for(kInt8), 1)
 template <bool kInt8>
 static cudaError_t launch_attention_t(const AttnMaps& maps, const AttnArgs& args,
                                       cudaStream_t stream) {
-  static int configured_mask = 0;
+  // devices whose kernel attributes are set (a set bit; set at most once
+  // per device, safely from several host threads)
+  static std::atomic<uint32_t> configured_mask{0u};
   constexpr uint32_t kSmem = smem_bytes(kInt8);
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 31 || !(configured_mask & (1 << dev))) {
+  if (dev >= 31 || !(configured_mask.load() & (1u << dev))) {
     e = cudaFuncSetAttribute(attn_fwd_kernel<kInt8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(kSmem));
     if (e != cudaSuccess) return e;
-    if (dev < 31) configured_mask |= 1 << dev;
+    if (dev < 31) configured_mask.fetch_or(1u << dev);
   }
   const unsigned grid = unsigned(args.n_full) + unsigned(args.n_split) * unsigned(args.chunks);
   attn_fwd_kernel<kInt8><<<grid, threads_for(kInt8), kSmem, stream>>>(
@@ -858,35 +844,6 @@ __global__ void __launch_bounds__(256) merge_kernel(const AttnArgs p) {
 cudaError_t launch_merge(const AttnArgs& args, cudaStream_t stream) {
   if (args.n_split <= 0) return cudaSuccess;
   merge_kernel<<<unsigned(args.n_split) * 32u, 256, 0, stream>>>(args);
-  return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------------------
-// exp2 evaluators, for testing them against each other
-// ---------------------------------------------------------------------------
-
-__global__ void exp2_eval_kernel(const float* x, float* y_poly, float* y_mufu, int64_t n) {
-  const int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 2;
-  if (i + 1 < n) {
-    float a, b;
-    exp2_poly2(x[i], x[i + 1], a, b);
-    y_poly[i] = a;
-    y_poly[i + 1] = b;
-    y_mufu[i] = ex2(x[i]);
-    y_mufu[i + 1] = ex2(x[i + 1]);
-  } else if (i < n) {
-    float a, b;
-    exp2_poly2(x[i], x[i], a, b);
-    y_poly[i] = a;
-    y_mufu[i] = ex2(x[i]);
-  }
-}
-
-cudaError_t launch_exp2_eval(const float* x, float* y_poly, float* y_mufu, int64_t n,
-                             cudaStream_t stream) {
-  if (n <= 0) return cudaSuccess;
-  const int64_t threads = (n + 1) / 2;
-  exp2_eval_kernel<<<unsigned((threads + 255) / 256), 256, 0, stream>>>(x, y_poly, y_mufu, n);
   return cudaGetLastError();
 }
 

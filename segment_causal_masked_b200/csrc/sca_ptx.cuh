@@ -79,6 +79,23 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
   }
 }
 
+// Time a CTA gives the loads and products it armed itself to land before it
+// exits (see wait_drain); independent of the pipeline waits' limit.
+constexpr unsigned long long kDrainTimeoutNs = 2000000000ull;
+
+// Wait for a phase the CTA armed itself (its own TMA loads, or a commit after
+// its own MMAs) before it may free its tensor memory and exit. Unlike
+// wait_bounded this ignores the abort flag, so an aborted CTA still lets
+// every copy and product in flight complete; it gives up only after
+// kDrainTimeoutNs. Returns whether the phase completed.
+__device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_ns() - t0 > kDrainTimeoutNs) return false;
+  return true;
+}
+
 // One try first; the bounded polling loop only when the phase is not complete
 // yet. (Everything is inlined: a shared out-of-line callee would stop ptxas
 // from giving the warpgroups different register budgets.)
@@ -289,34 +306,6 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
-}
-
-// 2^x on the FMA pipe, for finite x <= 8 (Cody-Waite range reduction):
-// x = j + f with j = rint(x) and f in [-1/2, 1/2]; 2^f from a cubic fitted
-// for minimax relative error on [-1/2, 1/2] by csrc/fit_exp2.py (Remez
-// exchange, 7.5e-5 after rounding the coefficients to float32); 2^j is added
-// to the exponent field. x is clamped at -126 so the exponent stays in range;
-// below that the result is a negligible value near 2^-126 (not 0), so this is
-// only used where no score is -inf (FULL tiles).
-constexpr float kExp2C0 = 0x1.fff692p-1f;
-constexpr float kExp2C1 = 0x1.62f31ap-1f;
-constexpr float kExp2C2 = 0x1.f0de1ap-3f;
-constexpr float kExp2C3 = 0x1.c3f76p-5f;
-constexpr float kRoundMagic = 12582912.f;  // 1.5 * 2^23: adding it leaves rint(x) in the low bits
-
-__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
-  const uint64_t x = f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
-  const uint64_t t = add2(x, f2(kRoundMagic, kRoundMagic));
-  const uint64_t j = add2(t, f2(-kRoundMagic, -kRoundMagic));
-  const uint64_t f = fma2(j, f2(-1.f, -1.f), x);
-  uint64_t p = fma2(f2(kExp2C3, kExp2C3), f, f2(kExp2C2, kExp2C2));
-  p = fma2(p, f, f2(kExp2C1, kExp2C1));
-  p = fma2(p, f, f2(kExp2C0, kExp2C0));
-  float p0, p1, t0, t1;
-  unf2(p, p0, p1);
-  unf2(t, t0, t1);
-  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

@@ -41,8 +41,8 @@ EXPORTED = (
     "sca_attn_workspace_bytes", "sca_attn_plan", "sca_attn_plan_for_sms",
     "sca_attn_int8_scratch_bytes",
     "sca_action_causal_attn_bwd", "sca_attn_bwd_workspace_bytes",
-    "sca_set_split_override",
-    "sca_last_error", "sca_debug_bounded_wait", "sca_debug_exp2",
+    "sca_set_split_override", "sca_set_pipeline_timeout_ns",
+    "sca_last_error", "sca_read_device_status", "sca_debug_bounded_wait",
 )
 
 
@@ -103,9 +103,10 @@ _SIGS = {
     "sca_attn_plan": [_P, _i32, _pi32, _pi32, _pi32],
     "sca_attn_plan_for_sms": [_P, _i32, _i32, _pi32, _pi32, _pi32, ctypes.POINTER(ctypes.c_uint64)],
     "sca_set_split_override": [_i32],
+    "sca_set_pipeline_timeout_ns": [_i64],
     "sca_last_error": [],
+    "sca_read_device_status": [_P, _P],
     "sca_debug_bounded_wait": [_P, _i64, _P],
-    "sca_debug_exp2": [_P, _P, _P, _i64, _P],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -369,10 +370,10 @@ def action_causal_attn_fwd_static_ws(cache: Optional[KVCache], md: Metadata, hea
     """Same result as ``action_causal_attn_fwd`` with a workspace, for callers
     that must not allocate: the key-split scratch comes from a fixed array of
     ``STATIC_WORKSPACE_BYTES`` inside the library (shared by all calls, so
-    calls must not overlap on the GPU). Raises ``ScaError`` with
-    ``ERR_CAPACITY`` when the call would need more scratch than that. The
-    first call on a device looks the array up and should precede any stream
-    capture."""
+    calls must not overlap on the GPU). An automatic split plan that needs
+    more runs unsplit; a forced split (``set_split_override``) that needs
+    more raises ``ScaError`` with ``ERR_CAPACITY``. The first call on a
+    device looks the array up and should precede any stream capture."""
     _check(_lib.sca_action_causal_attn_fwd_static_ws(
         cache.handle if cache is not None else None, md.handle, int(heads), _ptr(q), _ptr(k_cur),
         _ptr(v_cur), _ptr(o), _ptr(lse), float(softmax_scale), _ptr(dev_status), _stream(stream)))
@@ -435,15 +436,23 @@ def attn_plan_for_sms(md: Metadata, heads: int, sms: int) -> dict:
 
 
 def set_split_override(chunks: int) -> None:
-    """0 = automatic split plan, 1 = never split, k >= 2 = split the tail into k chunks."""
+    """0 = automatic split plan, 1 = never split, k >= 2 = split the tail into
+    k chunks; for calls made from the calling thread."""
     _check(_lib.sca_set_split_override(int(chunks)))
+
+
+def read_device_status(dev_status, stream=None) -> int:
+    """The status word after the stream's queued work: 0, else raises
+    ``ScaError`` with the code a kernel stored there."""
+    _check(_lib.sca_read_device_status(_ptr(dev_status), _stream(stream)))
+    return OK
+
+
+def set_pipeline_timeout_ns(ns: int) -> None:
+    """Limit of the kernels' pipeline waits for calls from the calling thread
+    (default 2 s; 0 exercises the abort path)."""
+    _check(_lib.sca_set_pipeline_timeout_ns(int(ns)))
 
 
 def debug_bounded_wait(dev_status, timeout_ns: int, stream=None) -> None:
     _check(_lib.sca_debug_bounded_wait(_ptr(dev_status), int(timeout_ns), _stream(stream)))
-
-
-def debug_exp2(x, y_poly, y_mufu, stream=None) -> None:
-    """The kernel's two exp2 evaluators on a float32 device tensor x."""
-    _check(_lib.sca_debug_exp2(_ptr(x), _ptr(y_poly), _ptr(y_mufu), int(x.numel()),
-                               _stream(stream)))

@@ -121,6 +121,39 @@ def test_backward_rejects_cache_and_missing_workspace():
     assert e.value.code == sca.ERR_CAPACITY
 
 
+def test_pipeline_timeout_aborts_the_backward_cleanly():
+    """The backward's three kernels with the pipeline-wait limit at 0: the
+    call reports SCA_ERR_DEVICE_TIMEOUT, every CTA drains its own loads and
+    products before it exits, and with the default limit restored the next
+    backward on the same handles matches the oracle."""
+    p = _packed("packed-14", 21, 14, heads=4)
+    b = Bwd(p, 85)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dq, dk, dv = (torch.empty_like(b.s.q) for _ in range(3))
+    ws = torch.empty(sca.attn_bwd_workspace_bytes(b.s.md, p.heads), dtype=torch.uint8,
+                     device="cuda")
+    try:
+        sca.set_pipeline_timeout_ns(0)
+        # a wait whose phase completes within the hardware's own try-wait
+        # window does not time out even at 0: repeat until one call gives up
+        for _ in range(5):
+            sca.action_causal_attn_bwd(b.s.md, p.heads, b.s.q, b.s.k_cur, b.s.v_cur, b.o, b.lse,
+                                       b.d_o, dq, dk, dv, p.softmax_scale, ws, None, st)
+            torch.cuda.synchronize()
+            if int(st.item()) != 0:
+                break
+    finally:
+        sca.set_pipeline_timeout_ns(2_000_000_000)
+    assert int(st.item()) == sca.ERR_DEVICE_TIMEOUT
+    x = torch.ones(4, device="cuda")
+    assert float((x * 2).sum().item()) == 8.0
+    dq, dk, dv = b.backward()
+    q, k, v, d_o = b.oracle_inputs()
+    refs = obwd.attention_backward(orule.Layout.of(p), q, k, v, d_o, p.softmax_scale)
+    for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), refs):
+        _check(name, got, ref)
+
+
 @pytest.mark.slow
 def test_backward_packed_360k_sampled_rows_and_identities():
     p = W.packed_360k()
