@@ -77,12 +77,13 @@ def test_split_keys_and_merge(p, chunks):
     q, k, v = oracle_inputs(inputs)
     o_ref, lse_ref = oattn.attention(orule.Layout.of(p), q, k, v, p.softmax_scale)
     compare(o2, l2, o_ref, lse_ref)
-    # The split only reorders fp32 sums (the same exponentials and products):
-    # after the bf16 rounding of O an element may move by one bf16 ulp
-    # (at most 2^-7 of its magnitude), plus the fp32 noise of elements near 0;
-    # LSE by a few fp32 ulps (measured at most 3.8e-6 on these layouts).
-    a, b = o1.float(), o2.float()
-    assert torch.all((a - b).abs() <= torch.maximum(a.abs(), b.abs()) * 2.0 ** -7 + 2e-5)
+    # A key chunk rounds its P to bf16 relative to its own running maximum, so
+    # the two calls round P differently (2^-9 relative each): with |v| < 4.6
+    # here that bounds |dO| near 2^-8 * 4.6 = 0.018 before O's own bf16
+    # rounding; measured at most 0.0156 (one ulp at [2, 4)) at this sharpness.
+    # LSE sums the unrounded p in fp32: it moves by a few fp32 ulps only
+    # (measured at most 3.8e-6 over 108 split / sharpness / seed cases).
+    assert (o1.float() - o2.float()).abs().max().item() <= 1.6e-2
     assert (l1 - l2).abs().max().item() <= 1e-5
 
 
