@@ -147,6 +147,39 @@ __device__ __forceinline__ void ds_pairs(const float (&s)[32], const float (&dp)
   }
 }
 
+// The two halves of ds_pairs, for a caller that stores P before it has dP:
+// p = 2^(s · scale_log2 − L), masked like ds_pairs, in place, with its bf16
+// pairs in pw ...
+template <bool kFull>
+__device__ __forceinline__ void p_pairs(float (&s)[32], uint32_t vis, uint64_t c2,
+                                        const uint64_t* nl2, uint32_t (&pw)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float x0, x1;
+    unf2(fma2(f2(s[2 * i], s[2 * i + 1]), c2, nl2[i]), x0, x1);
+    float p0 = ex2(x0), p1 = ex2(x1);
+    if (!kFull) {
+      p0 = ((vis >> (2 * i)) & 1u) ? p0 : 0.f;
+      p1 = ((vis >> (2 * i + 1)) & 1u) ? p1 : 0.f;
+    }
+    s[2 * i] = p0;
+    s[2 * i + 1] = p1;
+    pw[i] = pack_bf16(p0, p1);
+  }
+}
+
+// ... and then dS = P ∘ (dP − D) as bf16 pairs (the same operations, in the
+// same order, as ds_pairs)
+__device__ __forceinline__ void ds_from_p(const float (&p)[32], const float (&dp)[32],
+                                          const uint64_t* nd2, uint32_t (&dsw)[16]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float d0, d1;
+    unf2(mul2(f2(p[2 * i], p[2 * i + 1]), add2(f2(dp[2 * i], dp[2 * i + 1]), nd2[i])), d0, d1);
+    dsw[i] = pack_bf16(d0, d1);
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -493,8 +526,9 @@ constexpr uint32_t kKOffK = 0, kKOffV = kBTile, kKOffStage = 2 * kBTile;
 constexpr uint32_t kKStage = 2 * kBTile + 1024;  // Q, dO, D[128], L[128]
 constexpr int kKStages = 2;
 constexpr uint32_t kKBarKV = 0, kKBarF = 1, kKBarE = kKBarF + kKStages, kKBarST = kKBarE + kKStages,
-                   kKBarDPT = kKBarST + 1, kKBarRD = kKBarDPT + 1, kKBarDS = kKBarRD + 1,
-                   kKBarDone = kKBarDS + 1, kKBarDrain = kKBarDone + 1, kKNumBars = kKBarDrain + 1;
+                   kKBarDPT = kKBarST + 1, kKBarRD = kKBarDPT + 1, kKBarPR = kKBarRD + 1,
+                   kKBarDS = kKBarPR + 1, kKBarDone = kKBarDS + 1, kKBarDrain = kKBarDone + 1,
+                   kKNumBars = kKBarDrain + 1;
 constexpr uint32_t kKOffBar = kKOffStage + kKStages * kKStage;
 constexpr uint32_t kKOffCtl = kKOffBar + kKNumBars * 8;
 constexpr uint32_t kKOffSlot = kKOffCtl + 16;
@@ -533,6 +567,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     mbar_init(bar(kKBarST), 1);
     mbar_init(bar(kKBarDPT), 1);
     mbar_init(bar(kKBarRD), 256);
+    mbar_init(bar(kKBarPR), 256);
     mbar_init(bar(kKBarDS), 256);
     mbar_init(bar(kKBarDone), 1);
     mbar_init(bar(kKBarDrain), 1);
@@ -614,11 +649,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
           tc_fence_after();
           issue_dp(i + 1);
         }
+        const uint32_t st = sbase + stage(i);
+        // dV += Pᵀ dO as soon as Pᵀ is stored (it runs while the elementwise
+        // warps form dSᵀ), then dK += dSᵀ Q (B MN-major: rows are queries)
+        if (!(ok = wait_bar(bar(kKBarPR), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns))) break;
+        tc_fence_after();
+        mma_ts8_blocks(tDV, tSt, desc_mnmajor(st + kBTile), kIdescPV, i > 0 ? 1u : 0u);
         if (!(ok = wait_bar(bar(kKBarDS), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns))) break;
         tc_fence_after();
-        const uint32_t st = sbase + stage(i);
-        // dV += Pᵀ dO, dK += dSᵀ Q (B MN-major: rows are queries)
-        mma_ts8_blocks(tDV, tSt, desc_mnmajor(st + kBTile), kIdescPV, i > 0 ? 1u : 0u);
         mma_ts8_blocks(tDK, tSt + 64, desc_mnmajor(st), kIdescPV, i > 0 ? 1u : 0u);
         mma_commit(bar(kKBarE + i % kKStages));
         if (i + 1 < n) issue_s(i + 1);
@@ -684,24 +722,40 @@ __global__ void __launch_bounds__(kBThreads, 1)
       // dSᵀ to [64 + 32 half + 16 b, +16): only columns this thread has read.
       // (16-byte broadcast loads: four columns' -D or -L per load)
       const ulonglong2* ndl = reinterpret_cast<const ulonglong2*>(smem + stage(i) + 2 * kBTile);
+      // Pᵀ first: dV += Pᵀ dO starts on its barrier while dSᵀ is formed
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         const int cb = 64 * b + 32 * half;
-        uint64_t nd2[16], nl2[16];
+        uint64_t nl2[16];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const ulonglong2 d = ndl[cb / 4 + k], l = ndl[32 + cb / 4 + k];
-          nd2[2 * k] = d.x;
-          nd2[2 * k + 1] = d.y;
+          const ulonglong2 l = ndl[32 + cb / 4 + k];
           nl2[2 * k] = l.x;
           nl2[2 * k + 1] = l.y;
         }
-        const float(&sb)[32] = *reinterpret_cast<const float(*)[32]>(s + 32 * b);
-        const float(&dpb)[32] = *reinterpret_cast<const float(*)[32]>(dp + 32 * b);
-        uint32_t pw[16], dsw[16];
-        if (cls == SCA_TILE_FULL) ds_pairs<true>(sb, dpb, 0u, c2, nl2, nd2, dsw, pw);
-        else ds_pairs<false>(sb, dpb, vis[b], c2, nl2, nd2, dsw, pw);
+        float(&sb)[32] = *reinterpret_cast<float(*)[32]>(s + 32 * b);
+        uint32_t pw[16];
+        if (cls == SCA_TILE_FULL) p_pairs<true>(sb, 0u, c2, nl2, pw);
+        else p_pairs<false>(sb, vis[b], c2, nl2, pw);
         tmem_st16(tSt + lane_base + 32 * half + 16 * b, pw);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kKBarPR));
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        const int cb = 64 * b + 32 * half;
+        uint64_t nd2[16];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const ulonglong2 d = ndl[cb / 4 + k];
+          nd2[2 * k] = d.x;
+          nd2[2 * k + 1] = d.y;
+        }
+        const float(&pb)[32] = *reinterpret_cast<const float(*)[32]>(s + 32 * b);
+        const float(&dpb)[32] = *reinterpret_cast<const float(*)[32]>(dp + 32 * b);
+        uint32_t dsw[16];
+        ds_from_p(pb, dpb, nd2, dsw);
         tmem_st16(tSt + lane_base + 64 + 32 * half + 16 * b, dsw);
       }
       tmem_wait_st();

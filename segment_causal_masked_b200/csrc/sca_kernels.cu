@@ -541,14 +541,18 @@ __global__ void __launch_bounds__(threads_for(kInt8), 1)
       // a tile of the pair that sees nothing of key tile j gets neither its
       // S nor its P V; its barriers still complete (a commit with nothing
       // new arrives once the earlier MMAs are done)
-      auto live = [&](int j, int t) { return ((list[j] >> (24 + 2 * t)) & 3u) != SCA_TILE_EMPTY; };
+      // (schedule entries of key tiles j and j + 1 stay in registers; the
+      // entry of j + 2 is fetched one step ahead, off the issue path)
+      auto live = [&](uint32_t e, int t) { return ((e >> (24 + 2 * t)) & 3u) != SCA_TILE_EMPTY; };
+      uint32_t e_cur = list[0];
+      uint32_t e_nxt = n_iter > 1 ? list[1] : 0u;
       bool acc0 = false, acc1 = false;  // has O_t received a P V yet
       bool ok = wait_bar(bar(kBarQ), 0, ctl, p.status, p.timeout_ns) && wait_full(0);
       if (ok) {
         tc_fence_after();
-        if (live(0, 0)) issue_qk(tS0, sQ0, stage_of(0));
+        if (live(e_cur, 0)) issue_qk(tS0, sQ0, stage_of(0));
         mma_commit(bar(kBarS + 0));
-        if (live(0, 1)) issue_qk(tS1, sQ1, stage_of(0));
+        if (live(e_cur, 1)) issue_qk(tS1, sQ1, stage_of(0));
         mma_commit(bar(kBarS + 1));
         mma_commit(bar(kBarEmpty + 0));
       }
@@ -556,31 +560,34 @@ __global__ void __launch_bounds__(threads_for(kInt8), 1)
         const int itV = 2 * j + 1, itK = 2 * j + 2;
         const uint32_t ph = uint32_t(j) & 1u;
         const bool more = j + 1 < n_iter;
-        ok = wait_full(itV) && wait_bar(bar(kBarP + 0), ph, ctl, p.status, p.timeout_ns);
+        const uint32_t e_after = j + 2 < n_iter ? list[j + 2] : 0u;
+        // K of the next tile first, so that P V and the next S go out back to back
+        ok = wait_full(itV) && (!more || wait_full(itK)) &&
+             wait_bar(bar(kBarP + 0), ph, ctl, p.status, p.timeout_ns);
         if (!ok) break;
         tc_fence_after();
-        if (live(j, 0)) {
+        if (live(e_cur, 0)) {
           issue_pv(tO0, tS0, stage_of(itV), acc0);
           acc0 = true;
         }
         if (more) {
-          if (!(ok = wait_full(itK))) break;
-          tc_fence_after();
-          if (live(j + 1, 0)) issue_qk(tS0, sQ0, stage_of(itK));
+          if (live(e_nxt, 0)) issue_qk(tS0, sQ0, stage_of(itK));
           mma_commit(bar(kBarS + 0));
         }
         if (!(ok = wait_bar(bar(kBarP + 1), ph, ctl, p.status, p.timeout_ns))) break;
         tc_fence_after();
-        if (live(j, 1)) {
+        if (live(e_cur, 1)) {
           issue_pv(tO1, tS1, stage_of(itV), acc1);
           acc1 = true;
         }
         mma_commit(bar(kBarEmpty + itV % kRing));
         if (more) {
-          if (live(j + 1, 1)) issue_qk(tS1, sQ1, stage_of(itK));
+          if (live(e_nxt, 1)) issue_qk(tS1, sQ1, stage_of(itK));
           mma_commit(bar(kBarS + 1));
           mma_commit(bar(kBarEmpty + itK % kRing));
         }
+        e_cur = e_nxt;
+        e_nxt = e_after;
       }
       mma_commit(bar(kBarO + 0));
       mma_commit(bar(kBarO + 1));

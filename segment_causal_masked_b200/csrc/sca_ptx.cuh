@@ -52,6 +52,25 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// try_wait that may suspend the thread until the phase completes, for at
+// most `ns` nanoseconds, instead of returning at once.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Longest a waiting thread sleeps in one try (it wakes as soon as the phase
+// completes). Sleeping instead of spinning leaves the issue slots of the
+// sub-partition to the warps that compute.
+constexpr uint32_t kSuspendNs = 2000;
+
 // Shared control block of one CTA.
 struct Ctl {
   int32_t abort;   // set by the first wait that times out
@@ -65,9 +84,12 @@ struct Ctl {
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile Ctl* ctl,
                                           int32_t* status, unsigned long long timeout_ns) {
   if (mbar_try_wait(bar, parity)) return true;
+  // a try never sleeps longer than the limit itself (at a limit of 0 the
+  // first incomplete try gives up)
+  const uint32_t nap = timeout_ns < kSuspendNs ? uint32_t(timeout_ns) : kSuspendNs;
   const uint64_t t0 = global_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait_suspend(bar, parity, nap)) return true;
     if ((i & 15u) == 0) {
       if (ctl->abort) return false;
       if (global_ns() - t0 > timeout_ns) {
@@ -91,7 +113,7 @@ constexpr unsigned long long kDrainTimeoutNs = 2000000000ull;
 __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
-  while (!mbar_try_wait(bar, parity))
+  while (!mbar_try_wait_suspend(bar, parity, kSuspendNs))
     if (global_ns() - t0 > kDrainTimeoutNs) return false;
   return true;
 }

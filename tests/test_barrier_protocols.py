@@ -165,11 +165,13 @@ def forward_int8(staged_tiles, ring, cslots, seed):
         for j in range(n):
             itv, itk = 2 * j + 1, 2 * j + 2
             more = j + 1 < n
+            # V of this tile and K of the next one before P of tile 0
             yield wait(("full", itv % ring), (itv // ring) & 1, itv // ring)
+            if more:
+                yield wait(("full", itk % ring), (itk // ring) & 1, itk // ring)
             yield wait(("P", 0), j & 1, j)
             use(itv)
             if more:
-                yield wait(("full", itk % ring), (itk // ring) & 1, itk // ring)
                 use(itk)
                 bars[("S", 0)].arrive()
             yield wait(("P", 1), j & 1, j)
@@ -288,7 +290,7 @@ def backward_dq(n, seed, ks=3, vs=2):
 def backward_dkdv(n, seed, stages=2):
     bars = {("F", s): Bar(1) for s in range(stages)}
     bars.update({("E", s): Bar(1) for s in range(stages)})
-    for name in ("KV", "ST", "DPT", "DONE", "RD", "DS"):
+    for name in ("KV", "ST", "DPT", "DONE", "RD", "PR", "DS"):
         bars[name] = Bar(1)
     stage, st, dpt = {}, {}, {}
 
@@ -317,7 +319,9 @@ def backward_dkdv(n, seed, stages=2):
                 assert stage[(i + 1) % stages] == i + 1 and dpt.get("read") == i
                 dpt["v"] = i + 1
                 bars["DPT"].arrive()
-            yield wait("DS", i & 1, i)
+            yield wait("PR", i & 1, i)  # dV from Pᵀ
+            assert st["v"] in (("P", i), ("PdS", i)) and stage[i % stages] == i
+            yield wait("DS", i & 1, i)  # dK from dSᵀ
             assert st["v"] == ("PdS", i) and stage[i % stages] == i
             stage[i % stages] = None
             bars[("E", i % stages)].arrive()
@@ -336,6 +340,10 @@ def backward_dkdv(n, seed, stages=2):
             yield wait("ST", i & 1, i)
             assert st["v"] == ("S", i) and stage[i % stages] == i
             yield ("work",)
+            st["v"] = ("P", i)
+            bars["PR"].arrive()
+            yield ("work",)
+            assert stage[i % stages] == i  # -D is still read from the stage
             st["v"] = ("PdS", i)
             bars["DS"].arrive()
         yield wait("DONE", 0, 0)
