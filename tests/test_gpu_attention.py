@@ -58,6 +58,30 @@ def test_attention_matches_oracle(p, q_scale):
     compare(o, lse, o_ref, lse_ref)
 
 
+@pytest.mark.parametrize("split", [0, 3], ids=["whole", "split3"])
+def test_large_score_jump_rescales_mid_row(split):
+    """Current keys 24 times the cached ones: a current-segment row first
+    sets its running max on cached tiles (scores of a few log2 units), then
+    meets tiles scoring more than 64 log2 units higher (exponentials against
+    the old max would overflow fp32). The running max moves, O and l are
+    rescaled, and O and LSE match the oracle, whole and split into key
+    chunks."""
+    p = W.small_session(heads=2)
+    inputs = W.make_inputs(p, 53)
+    inputs["k_cur"] = (inputs["k_cur"].float() * 24.0).to(torch.bfloat16)
+    s = GpuSession(p, inputs)
+    try:
+        sca.set_split_override(split)
+        o, lse = s.forward()
+    finally:
+        sca.set_split_override(0)
+    q, k, v = oracle_inputs(inputs)
+    scores = np.einsum("thd,shd->hts", q[:, :1], k[:, :1]) * p.softmax_scale / np.log(2.0)
+    assert scores.max() - scores[:, :, :p.n_cache_tokens].max() > 64  # the jump is there
+    o_ref, lse_ref = oattn.attention(orule.Layout.of(p), q, k, v, p.softmax_scale)
+    compare(o, lse, o_ref, lse_ref)
+
+
 @pytest.mark.parametrize("chunks", [2, 3, 7])
 @pytest.mark.parametrize("p", [W.small_session(), W.small_packed(seed=21, n_segments=14),
                                W.Problem("multi-pair", SMALL[7].cached, SMALL[7].current, heads=3)],
