@@ -520,22 +520,34 @@ __global__ void __launch_bounds__(kBThreads, 1)
 // dK and dV
 // ---------------------------------------------------------------------------
 
-// shared memory: K, V of the CTA's key tile, then 2 stages of (Q, dO, D, L)
-// of one query tile (65 KB each, so every tile stays 1024-aligned).
-constexpr uint32_t kKOffK = 0, kKOffV = kBTile, kKOffStage = 2 * kBTile;
-constexpr uint32_t kKStage = 2 * kBTile + 1024;  // Q, dO, D[128], L[128]
-constexpr int kKStages = 2;
-constexpr uint32_t kKBarKV = 0, kKBarF = 1, kKBarE = kKBarF + kKStages, kKBarST = kKBarE + kKStages,
-                   kKBarDPT = kKBarST + 1, kKBarRD = kKBarDPT + 1, kKBarPR = kKBarRD + 1,
-                   kKBarDS = kKBarPR + 1, kKBarDone = kKBarDS + 1, kKBarDrain = kKBarDone + 1,
-                   kKNumBars = kKBarDrain + 1;
-constexpr uint32_t kKOffBar = kKOffStage + kKStages * kKStage;
+// shared memory, from a 1024-aligned base: the barriers in the first 1 KB,
+// then K and V of the CTA's key tile, a ring of 3 Q tiles and a ring of 2
+// (dO tile, −D[128], −L[128]) stages (32 KB and 33 KB, so every tile stays
+// 1024-aligned): 227 KB, all a CTA may have, so there is no room to align
+// the base by hand and the kernel checks that it is aligned. Q_i is read by
+// Sᵀ_i and again by dK += dSᵀ_i Q_i a query tile later, while Sᵀ of the
+// next query tile is wanted early, so Q gets the deeper ring.
+constexpr uint32_t kKBarKV = 0, kKBarQF = 1, kKQSlots = 3, kKBarQE = kKBarQF + kKQSlots,
+                   kKOSlots = 2, kKBarOF = kKBarQE + kKQSlots, kKBarOE = kKBarOF + kKOSlots,
+                   kKBarST = kKBarOE + kKOSlots, kKBarDPT = kKBarST + 1, kKBarRD = kKBarDPT + 1,
+                   kKBarPR = kKBarRD + 1, kKBarDS = kKBarPR + 1, kKBarDone = kKBarDS + 1,
+                   kKBarDrain = kKBarDone + 1, kKNumBars = kKBarDrain + 1;
+constexpr uint32_t kKOffBar = 0;
 constexpr uint32_t kKOffCtl = kKOffBar + kKNumBars * 8;
 constexpr uint32_t kKOffSlot = kKOffCtl + 16;
-constexpr uint32_t kKSmem = kKOffSlot + 16 + 1024;
+constexpr uint32_t kKOffK = 1024, kKOffV = kKOffK + kBTile, kKOffQ = kKOffV + kBTile;
+constexpr uint32_t kKOStage = kBTile + 1024;  // dO, −D[128], −L[128]
+constexpr uint32_t kKOffO = kKOffQ + kKQSlots * kBTile;
+constexpr uint32_t kKSmem = kKOffO + kKOSlots * kKOStage;
+static_assert(kKOffSlot + 16 <= kKOffK, "the barriers fit the first 1 KB");
 static_assert(kKSmem <= 232448, "the dK/dV kernel must fit the 227 KB a CTA may use");
-static_assert(kKStage % 1024 == 0, "stages must keep the tiles 1024-aligned");
 
+// TMEM of the dK/dV kernel: two 128-column regions X and Y that swap roles
+// every query tile, then dV and dK. Query tile i computes Sᵀ_i into
+// region(i), overwrites it with Pᵀ_i (columns 0-63) and dSᵀ_i (64-127) for
+// dV and dK, and takes dPᵀ_i in region(i + 1); so Sᵀ_{i+1} may start as soon
+// as dPᵀ_i has been read out, while dV and dK of tile i still read region(i),
+// and dPᵀ_{i+1} goes into region(i) once they have.
 __global__ void __launch_bounds__(kBThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -547,12 +559,16 @@ __global__ void __launch_bounds__(kBThreads, 1)
   const uint32_t* list = p.kt_list + p.kt_ptr[ktile];
   const int n = p.kt_ptr[ktile + 1] - p.kt_ptr[ktile];
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {  // the layout needs a 1024-aligned base (uniform: all threads leave)
+    if (threadIdx.x == 0 && p.status) atomicExch(p.status, SCA_ERR_MISALIGNED);
+    return;
+  }
   auto bar = [&](uint32_t i) { return sbase + kKOffBar + 8 * i; };
-  auto stage = [&](int i) { return kKOffStage + uint32_t(i % kKStages) * kKStage; };
+  auto qslot = [&](int i) { return sbase + kKOffQ + uint32_t(i % kKQSlots) * kBTile; };
+  auto oslot = [&](int i) { return sbase + kKOffO + uint32_t(i % kKOSlots) * kKOStage; };
   volatile Ctl* ctl = reinterpret_cast<volatile Ctl*>(smem + kKOffCtl);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kKOffSlot);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -560,9 +576,13 @@ __global__ void __launch_bounds__(kBThreads, 1)
   if (threadIdx.x == 0) {
     ctl->abort = 0;
     mbar_init(bar(kKBarKV), 1);
-    for (int s = 0; s < kKStages; ++s) {
-      mbar_init(bar(kKBarF + s), 1);
-      mbar_init(bar(kKBarE + s), 1);
+    for (int s = 0; s < kKQSlots; ++s) {
+      mbar_init(bar(kKBarQF + s), 1);
+      mbar_init(bar(kKBarQE + s), 1);
+    }
+    for (int s = 0; s < kKOSlots; ++s) {
+      mbar_init(bar(kKBarOF + s), 1);
+      mbar_init(bar(kKBarOE + s), 1);
     }
     mbar_init(bar(kKBarST), 1);
     mbar_init(bar(kKBarDPT), 1);
@@ -584,12 +604,13 @@ __global__ void __launch_bounds__(kBThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tSt = tmem, tDPt = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
+  const uint32_t tDV = tmem + 256, tDK = tmem + 384;
+  auto region = [&](int i) { return tmem + uint32_t(i & 1) * 128; };
 
   if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kBRegsControl));
     if (warp == 8 && lane == 0) {
-      // ---------------------------------------------------------------- producer
+      // ------------------------------------------------------ producer: K, V, Q
       const int k0 = ktile * 128;
       mbar_expect_tx(bar(kKBarKV), 2 * kBTile);
       tma_load_3d(sbase + kKOffK, &tm_k, bar(kKBarKV), 0, head, k0);
@@ -598,68 +619,92 @@ __global__ void __launch_bounds__(kBThreads, 1)
       tma_load_3d(sbase + kKOffV + kBHalf, &tm_v, bar(kKBarKV), 64, head, k0);
       int i = 0;
       for (; i < n; ++i) {
-        const int s = i % kKStages;
-        if (!wait_bar(bar(kKBarE + s), (uint32_t(i / kKStages) & 1u) ^ 1u, ctl, p.status,
+        const int s = i % kKQSlots;
+        if (!wait_bar(bar(kKBarQE + s), (uint32_t(i / kKQSlots) & 1u) ^ 1u, ctl, p.status,
                       p.timeout_ns))
           break;
         const int q0 = int(list[i] & kPairTileMask) * 128;
-        const uint32_t st = sbase + stage(i), fb = bar(kKBarF + s);
-        mbar_expect_tx(fb, 2 * kBTile + 1024);
-        tma_load_3d(st, &tm_q, fb, 0, head, q0);
-        tma_load_3d(st + kBHalf, &tm_q, fb, 64, head, q0);
-        tma_load_3d(st + kBTile, &tm_do, fb, 0, head, q0);
-        tma_load_3d(st + kBTile + kBHalf, &tm_do, fb, 64, head, q0);
-        tma_load_2d(st + 2 * kBTile, &tm_dl, fb, q0, head);
-        tma_load_2d(st + 2 * kBTile + 512, &tm_dl, fb, q0, p.heads + head);
+        mbar_expect_tx(bar(kKBarQF + s), kBTile);
+        tma_load_3d(qslot(i), &tm_q, bar(kKBarQF + s), 0, head, q0);
+        tma_load_3d(qslot(i) + kBHalf, &tm_q, bar(kKBarQF + s), 64, head, q0);
       }
       // Drain, also after a normal end: every armed load lands before the
       // CTA can exit, even when a consumer gave up.
-      for (int i2 = i - kKStages < 0 ? 0 : i - kKStages; i2 < i; ++i2)
-        wait_drain(bar(kKBarF + i2 % kKStages), uint32_t(i2 / kKStages) & 1u);
+      for (int i2 = i - kKQSlots < 0 ? 0 : i - kKQSlots; i2 < i; ++i2)
+        wait_drain(bar(kKBarQF + i2 % kKQSlots), uint32_t(i2 / kKQSlots) & 1u);
       wait_drain(bar(kKBarKV), 0);
+    } else if (warp == 10 && lane == 0) {
+      // ------------------------------------------------------ producer: dO
+      int i = 0;
+      for (; i < n; ++i) {
+        const int s = i % kKOSlots;
+        if (!wait_bar(bar(kKBarOE + s), (uint32_t(i / kKOSlots) & 1u) ^ 1u, ctl, p.status,
+                      p.timeout_ns))
+          break;
+        const int q0 = int(list[i] & kPairTileMask) * 128;
+        mbar_expect_tx(bar(kKBarOF + s), kKOStage);
+        tma_load_3d(oslot(i), &tm_do, bar(kKBarOF + s), 0, head, q0);
+        tma_load_3d(oslot(i) + kBHalf, &tm_do, bar(kKBarOF + s), 64, head, q0);
+        tma_load_2d(oslot(i) + kBTile, &tm_dl, bar(kKBarOF + s), q0, head);
+        tma_load_2d(oslot(i) + kBTile + 512, &tm_dl, bar(kKBarOF + s), q0, p.heads + head);
+      }
+      for (int i2 = i - kKOSlots < 0 ? 0 : i - kKOSlots; i2 < i; ++i2)
+        wait_drain(bar(kKBarOF + i2 % kKOSlots), uint32_t(i2 / kKOSlots) & 1u);
     } else if (warp == 9 && lane == 0) {
       // ---------------------------------------------------------------- MMA
       const uint64_t dK = desc_kmajor(sbase + kKOffK), dV = desc_kmajor(sbase + kKOffV);
-      auto wait_f = [&](int i) {
-        return wait_bar(bar(kKBarF + i % kKStages), uint32_t(i / kKStages) & 1u, ctl, p.status,
+      auto wait_q = [&](int i) {
+        return wait_bar(bar(kKBarQF + i % kKQSlots), uint32_t(i / kKQSlots) & 1u, ctl, p.status,
                         p.timeout_ns);
       };
-      auto issue_s = [&](int i) {  // Sᵀ = K Qᵢᵀ
-        mma_qk8(tSt, dK, desc_kmajor(sbase + stage(i)), kIdescQK);
+      auto wait_o = [&](int i) {
+        return wait_bar(bar(kKBarOF + i % kKOSlots), uint32_t(i / kKOSlots) & 1u, ctl, p.status,
+                        p.timeout_ns);
+      };
+      auto issue_s = [&](int i) {  // Sᵀ_i = K Q_iᵀ into region(i)
+        mma_qk8(region(i), dK, desc_kmajor(qslot(i)), kIdescQK);
         mma_commit(bar(kKBarST));
       };
-      auto issue_dp = [&](int i) {  // dPᵀ = V dOᵢᵀ
-        mma_qk8(tDPt, dV, desc_kmajor(sbase + stage(i) + kBTile), kIdescQK);
+      auto issue_dp = [&](int i) {  // dPᵀ_i = V dO_iᵀ into region(i + 1)
+        mma_qk8(region(i + 1), dV, desc_kmajor(oslot(i)), kIdescQK);
         mma_commit(bar(kKBarDPT));
       };
       // K and V are always loaded: wait for them even with no query tile
-      bool ok = wait_bar(bar(kKBarKV), 0, ctl, p.status, p.timeout_ns) && (n == 0 || wait_f(0));
+      bool ok = wait_bar(bar(kKBarKV), 0, ctl, p.status, p.timeout_ns) &&
+                (n == 0 || (wait_q(0) && wait_o(0)));
       if (ok && n > 0) {
         tc_fence_after();
         issue_s(0);
         issue_dp(0);
       }
       for (int i = 0; ok && i < n; ++i) {
-        // the next dPᵀ as soon as this one has been read out (the elementwise
-        // warps write Pᵀ and dSᵀ into the Sᵀ columns only)
-        if (!(ok = wait_bar(bar(kKBarRD), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns))) break;
+        const bool more = i + 1 < n;
+        // dV += Pᵀ_i dO_i (B MN-major: rows are queries) as soon as Pᵀ_i is stored
+        if (!(ok = wait_bar(bar(kKBarPR), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns))) break;
         tc_fence_after();
-        if (i + 1 < n) {
-          if (!(ok = wait_f(i + 1))) break;
+        mma_ts8_blocks(tDV, region(i), desc_mnmajor(oslot(i)), kIdescPV, i > 0 ? 1u : 0u);
+        // Sᵀ_{i+1} into the other region as soon as dPᵀ_i has been read out
+        if (more) {
+          if (!(ok = wait_bar(bar(kKBarRD), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns) &&
+                     wait_q(i + 1)))
+            break;
+          tc_fence_after();
+          issue_s(i + 1);
+        }
+        // dK += dSᵀ_i Q_i
+        if (!(ok = wait_bar(bar(kKBarDS), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns))) break;
+        tc_fence_after();
+        mma_ts8_blocks(tDK, region(i) + 64, desc_mnmajor(qslot(i)), kIdescPV, i > 0 ? 1u : 0u);
+        mma_commit(bar(kKBarQE + i % kKQSlots));  // the last read of Q_i
+        // the dO stage too: dV has read dO_i and the elementwise warps their
+        // −D and −L before arriving on dSᵀ
+        mma_commit(bar(kKBarOE + i % kKOSlots));
+        // dPᵀ_{i+1} into region(i), after dV and dK have read it (in-order pipe)
+        if (more) {
+          if (!(ok = wait_o(i + 1))) break;
           tc_fence_after();
           issue_dp(i + 1);
         }
-        const uint32_t st = sbase + stage(i);
-        // dV += Pᵀ dO as soon as Pᵀ is stored (it runs while the elementwise
-        // warps form dSᵀ), then dK += dSᵀ Q (B MN-major: rows are queries)
-        if (!(ok = wait_bar(bar(kKBarPR), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns))) break;
-        tc_fence_after();
-        mma_ts8_blocks(tDV, tSt, desc_mnmajor(st + kBTile), kIdescPV, i > 0 ? 1u : 0u);
-        if (!(ok = wait_bar(bar(kKBarDS), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns))) break;
-        tc_fence_after();
-        mma_ts8_blocks(tDK, tSt + 64, desc_mnmajor(st), kIdescPV, i > 0 ? 1u : 0u);
-        mma_commit(bar(kKBarE + i % kKStages));
-        if (i + 1 < n) issue_s(i + 1);
       }
       mma_commit(bar(kKBarDone));
       mma_commit(bar(kKBarDrain));
@@ -694,42 +739,35 @@ __global__ void __launch_bounds__(kBThreads, 1)
           vis[1] |= run_bits32(a, b, 64 + 32 * half);
         }
       }
-      ok = wait_bar(bar(kKBarF + i % kKStages), uint32_t(i / kKStages) & 1u, ctl, p.status,
-                    p.timeout_ns) &&
-           wait_bar(bar(kKBarDPT), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns);
-      if (!__all_sync(0xFFFFFFFFu, ok)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      float dp[64], s[64];
-      tmem_ld32(tDPt + lane_base + 32 * half, dp);
-      tmem_ld32(tDPt + lane_base + 64 + 32 * half, dp + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(kKBarRD));  // dPᵀ is in registers: the next dPᵀ may overwrite it
+      const uint32_t tR = region(i) + lane_base, tD = region(i + 1) + lane_base;
+      // per query column −D and −L as pairs, from the dO stage; block b
+      // covers queries [64 b + 32 half, +32) (16-byte broadcast loads: four
+      // columns each)
+      const uint8_t* ost = smem + kKOffO + uint32_t(i % kKOSlots) * kKOStage;
+      const ulonglong2* ndq = reinterpret_cast<const ulonglong2*>(ost + kBTile);
+      const ulonglong2* nlq = reinterpret_cast<const ulonglong2*>(ost + kBTile + 512);
       if (!__all_sync(0xFFFFFFFFu, wait_bar(bar(kKBarST), uint32_t(i) & 1u, ctl, p.status,
-                                            p.timeout_ns))) {
+                                            p.timeout_ns) &&
+                                       wait_bar(bar(kKBarOF + i % kKOSlots),
+                                                uint32_t(i / kKOSlots) & 1u, ctl, p.status,
+                                                p.timeout_ns))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      tmem_ld32(tSt + lane_base + 32 * half, s);
-      tmem_ld32(tSt + lane_base + 64 + 32 * half, s + 32);
+      float s[64], dp[64];
+      tmem_ld32(tR + 32 * half, s);
+      tmem_ld32(tR + 64 + 32 * half, s + 32);
       tmem_wait_ld();
-      // per query column -D and -L as pairs; block b covers queries
-      // [64 b + 32 half, +32). Pᵀ goes to Sᵀ columns [32 half + 16 b, +16),
-      // dSᵀ to [64 + 32 half + 16 b, +16): only columns this thread has read.
-      // (16-byte broadcast loads: four columns' -D or -L per load)
-      const ulonglong2* ndl = reinterpret_cast<const ulonglong2*>(smem + stage(i) + 2 * kBTile);
-      // Pᵀ first: dV += Pᵀ dO starts on its barrier while dSᵀ is formed
+      // Pᵀ into region(i) columns [32 half + 16 b, +16), over scores this
+      // thread has read; dV += Pᵀ dO starts on its barrier
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         const int cb = 64 * b + 32 * half;
         uint64_t nl2[16];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const ulonglong2 l = ndl[32 + cb / 4 + k];
+          const ulonglong2 l = nlq[cb / 4 + k];
           nl2[2 * k] = l.x;
           nl2[2 * k + 1] = l.y;
         }
@@ -737,18 +775,30 @@ __global__ void __launch_bounds__(kBThreads, 1)
         uint32_t pw[16];
         if (cls == SCA_TILE_FULL) p_pairs<true>(sb, 0u, c2, nl2, pw);
         else p_pairs<false>(sb, vis[b], c2, nl2, pw);
-        tmem_st16(tSt + lane_base + 32 * half + 16 * b, pw);
+        tmem_st16(tR + 32 * half + 16 * b, pw);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kKBarPR));
+      if (!__all_sync(0xFFFFFFFFu, wait_bar(bar(kKBarDPT), uint32_t(i) & 1u, ctl, p.status,
+                                            p.timeout_ns))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      tmem_ld32(tD + 32 * half, dp);
+      tmem_ld32(tD + 64 + 32 * half, dp + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(kKBarRD));  // dPᵀ is in registers: Sᵀ of the next tile may overwrite it
+      // dSᵀ into region(i) columns [64 + 32 half + 16 b, +16)
 #pragma unroll
       for (int b = 0; b < 2; ++b) {
         const int cb = 64 * b + 32 * half;
         uint64_t nd2[16];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const ulonglong2 d = ndl[cb / 4 + k];
+          const ulonglong2 d = ndq[cb / 4 + k];
           nd2[2 * k] = d.x;
           nd2[2 * k + 1] = d.y;
         }
@@ -756,7 +806,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
         const float(&dpb)[32] = *reinterpret_cast<const float(*)[32]>(dp + 32 * b);
         uint32_t dsw[16];
         ds_from_p(pb, dpb, nd2, dsw);
-        tmem_st16(tSt + lane_base + 64 + 32 * half + 16 * b, dsw);
+        tmem_st16(tR + 64 + 32 * half + 16 * b, dsw);
       }
       tmem_wait_st();
       tc_fence_before();

@@ -287,68 +287,104 @@ def backward_dq(n, seed, ks=3, vs=2):
     run({"producer": producer(), "mma": mma(), "elementwise": elementwise()}, bars, seed)
 
 
-def backward_dkdv(n, seed, stages=2):
-    bars = {("F", s): Bar(1) for s in range(stages)}
-    bars.update({("E", s): Bar(1) for s in range(stages)})
-    for name in ("KV", "ST", "DPT", "DONE", "RD", "PR", "DS"):
+def backward_dkdv(n, seed, qslots=3, oslots=2):
+    """The dK/dV kernel: a Q ring (3) and a ring of dO stages with −D, −L (2),
+    each with its own loader; TMEM regions X, Y swap roles per query tile:
+    Sᵀ_i into region i % 2, then Pᵀ_i and dSᵀ_i over it; dPᵀ_i into region
+    (i + 1) % 2. Region contents are tracked, and every product or store
+    checks what it overwrites."""
+    bars = {}
+    for s in range(qslots):
+        bars[("QF", s)], bars[("QE", s)] = Bar(1), Bar(1)
+    for s in range(oslots):
+        bars[("OF", s)], bars[("OE", s)] = Bar(1), Bar(1)
+    for name in ("KV", "ST", "DPT", "DONE"):
         bars[name] = Bar(1)
-    stage, st, dpt = {}, {}, {}
+    for name in ("RD", "PR", "DS"):  # the elementwise warps (one arrival stands for 256)
+        bars[name] = Bar(1)
+    qring, oring, reg, dp_read = {}, {}, {0: None, 1: None}, set()
 
-    def producer():
+    def producer_q():
         bars["KV"].expect(1)
         yield ("copy", "KV", 1)
         for i in range(n):
-            yield wait(("E", i % stages), ((i // stages) & 1) ^ 1, i // stages - 1)
-            assert stage.get(i % stages) is None
-            stage[i % stages] = i
-            bars[("F", i % stages)].expect(1)
-            yield ("copy", ("F", i % stages), 1)
+            s = i % qslots
+            yield wait(("QE", s), ((i // qslots) & 1) ^ 1, i // qslots - 1)
+            assert qring.get(s) is None, "Q slot refilled while in use"
+            qring[s] = i
+            bars[("QF", s)].expect(1)
+            yield ("copy", ("QF", s), 1)
+
+    def producer_o():
+        for i in range(n):
+            s = i % oslots
+            yield wait(("OE", s), ((i // oslots) & 1) ^ 1, i // oslots - 1)
+            assert oring.get(s) is None, "dO slot refilled while in use"
+            oring[s] = i
+            bars[("OF", s)].expect(1)
+            yield ("copy", ("OF", s), 1)
+
+    def issue_s(i):  # Sᵀ_i into region i % 2, over dPᵀ_{i-1} once it has been read out
+        assert qring.get(i % qslots) == i
+        cur = reg[i % 2]
+        assert cur is None or (cur == ("dP", i - 1) and i - 1 in dp_read), ("S over live", cur)
+        reg[i % 2] = ("S", i)
+        bars["ST"].arrive()
+
+    def issue_dp(i):  # dPᵀ_i into region (i + 1) % 2, after dV and dK of tile i - 1
+        assert oring.get(i % oslots) == i
+        cur = reg[(i + 1) % 2]
+        assert cur is None or cur == ("PdS", i - 1), ("dP over live", cur)
+        reg[(i + 1) % 2] = ("dP", i)
+        bars["DPT"].arrive()
 
     def mma():
+        # products are modelled at issue (the tensor pipe runs them in order)
         yield wait("KV", 0, 0)
         if n:
-            yield wait(("F", 0), 0, 0)
-            st["v"] = ("S", 0)
-            bars["ST"].arrive()
-            dpt["v"] = 0
-            bars["DPT"].arrive()
+            yield wait(("QF", 0), 0, 0)
+            yield wait(("OF", 0), 0, 0)
+            issue_s(0)
+            issue_dp(0)
         for i in range(n):
-            yield wait("RD", i & 1, i)
-            if i + 1 < n:
-                yield wait(("F", (i + 1) % stages), ((i + 1) // stages) & 1, (i + 1) // stages)
-                assert stage[(i + 1) % stages] == i + 1 and dpt.get("read") == i
-                dpt["v"] = i + 1
-                bars["DPT"].arrive()
-            yield wait("PR", i & 1, i)  # dV from Pᵀ
-            assert st["v"] in (("P", i), ("PdS", i)) and stage[i % stages] == i
-            yield wait("DS", i & 1, i)  # dK from dSᵀ
-            assert st["v"] == ("PdS", i) and stage[i % stages] == i
-            stage[i % stages] = None
-            bars[("E", i % stages)].arrive()
-            if i + 1 < n:
-                st["v"] = ("S", i + 1)
-                bars["ST"].arrive()
+            more = i + 1 < n
+            yield wait("PR", i & 1, i)  # dV from Pᵀ_i and dO_i
+            assert reg[i % 2] in (("P", i), ("PdS", i)) and oring.get(i % oslots) == i
+            if more:
+                yield wait("RD", i & 1, i)
+                yield wait(("QF", (i + 1) % qslots), ((i + 1) // qslots) & 1, (i + 1) // qslots)
+                issue_s(i + 1)
+            yield wait("DS", i & 1, i)  # dK from dSᵀ_i and Q_i
+            assert reg[i % 2] == ("PdS", i) and qring.get(i % qslots) == i
+            qring[i % qslots] = None
+            bars[("QE", i % qslots)].arrive()
+            oring[i % oslots] = None  # dV and the elementwise warps are done with the dO stage
+            bars[("OE", i % oslots)].arrive()
+            if more:
+                yield wait(("OF", (i + 1) % oslots), ((i + 1) // oslots) & 1, (i + 1) // oslots)
+                issue_dp(i + 1)
         bars["DONE"].arrive()
 
     def elementwise():
         for i in range(n):
-            yield wait(("F", i % stages), (i // stages) & 1, i // stages)
-            yield wait("DPT", i & 1, i)
-            assert dpt["v"] == i
-            dpt["read"] = i
-            bars["RD"].arrive()
             yield wait("ST", i & 1, i)
-            assert st["v"] == ("S", i) and stage[i % stages] == i
+            yield wait(("OF", i % oslots), (i // oslots) & 1, i // oslots)
+            assert reg[i % 2] == ("S", i) and oring.get(i % oslots) == i  # −L from the stage
             yield ("work",)
-            st["v"] = ("P", i)
+            reg[i % 2] = ("P", i)  # Pᵀ over the scores just read
             bars["PR"].arrive()
+            yield wait("DPT", i & 1, i)
+            assert reg[(i + 1) % 2] == ("dP", i)
+            dp_read.add(i)
+            bars["RD"].arrive()
             yield ("work",)
-            assert stage[i % stages] == i  # -D is still read from the stage
-            st["v"] = ("PdS", i)
+            assert reg[i % 2] == ("P", i) and oring.get(i % oslots) == i  # −D from the stage
+            reg[i % 2] = ("PdS", i)
             bars["DS"].arrive()
         yield wait("DONE", 0, 0)
 
-    run({"producer": producer(), "mma": mma(), "elementwise": elementwise()}, bars, seed)
+    run({"producer_q": producer_q(), "producer_o": producer_o(), "mma": mma(),
+         "elementwise": elementwise()}, bars, seed)
 
 
 def test_backward_dq_pipeline():
@@ -394,3 +430,29 @@ def test_missing_prefix_wait_would_be_caught():
             for n_staged in range(1, n):
                 for seed in range(8):
                     scope["forward_int8"]([True] * n_staged + [False] * (n - n_staged), 2, 5, seed)
+
+
+@pytest.mark.parametrize("mutation", ["no read-out wait before the next S", "next dP before dS"])
+def test_dkdv_region_hazards_would_be_caught(mutation):
+    """The dK/dV model is sharp: Sᵀ of the next query tile issued before dPᵀ
+    was read out of its region, or dPᵀ of the next tile issued before dK had
+    read dSᵀ, is reported in some interleaving."""
+    import inspect
+    src = inspect.getsource(backward_dkdv)
+    if mutation.startswith("no read-out"):
+        src = src.replace('                yield wait("RD", i & 1, i)\n', '')
+    else:
+        src = src.replace(
+            '            yield wait("DS", i & 1, i)  # dK from dSᵀ_i and Q_i',
+            '            if more:\n'
+            '                yield wait(("OF", (i + 1) % oslots), ((i + 1) // oslots) & 1, (i + 1) // oslots)\n'
+            '                issue_dp(i + 1)\n'
+            '                more = False\n'
+            '            yield wait("DS", i & 1, i)  # dK from dSᵀ_i and Q_i')
+    assert src != inspect.getsource(backward_dkdv)
+    scope = dict(globals())
+    exec(src, scope)
+    with pytest.raises(AssertionError):
+        for n in range(2, 8):
+            for seed in range(40):
+                scope["backward_dkdv"](n, seed)
