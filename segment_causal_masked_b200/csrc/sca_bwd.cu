@@ -679,11 +679,12 @@ __global__ void __launch_bounds__(kBThreads, 1)
       }
       for (int i = 0; ok && i < n; ++i) {
         const bool more = i + 1 < n;
-        // dV += Pᵀ_i dO_i (B MN-major: rows are queries) as soon as Pᵀ_i is stored
+        // Pᵀ_i stored (waited first: the elementwise warps cannot store Pᵀ_{i+1}
+        // before Sᵀ_{i+1} below, so this barrier is never a phase ahead)
         if (!(ok = wait_bar(bar(kKBarPR), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns))) break;
-        tc_fence_after();
-        mma_ts8_blocks(tDV, region(i), desc_mnmajor(oslot(i)), kIdescPV, i > 0 ? 1u : 0u);
-        // Sᵀ_{i+1} into the other region as soon as dPᵀ_i has been read out
+        // Sᵀ_{i+1} into the other region as soon as dPᵀ_i has been read out,
+        // ahead of dV in the pipe: the next query tile's elementwise work
+        // waits on it, while dV is needed only before the next dV
         if (more) {
           if (!(ok = wait_bar(bar(kKBarRD), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns) &&
                      wait_q(i + 1)))
@@ -691,6 +692,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
           tc_fence_after();
           issue_s(i + 1);
         }
+        // dV += Pᵀ_i dO_i (B MN-major: rows are queries)
+        tc_fence_after();
+        mma_ts8_blocks(tDV, region(i), desc_mnmajor(oslot(i)), kIdescPV, i > 0 ? 1u : 0u);
         // dK += dSᵀ_i Q_i
         if (!(ok = wait_bar(bar(kKBarDS), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns))) break;
         tc_fence_after();

@@ -348,12 +348,13 @@ def backward_dkdv(n, seed, qslots=3, oslots=2):
             issue_dp(0)
         for i in range(n):
             more = i + 1 < n
-            yield wait("PR", i & 1, i)  # dV from Pᵀ_i and dO_i
-            assert reg[i % 2] in (("P", i), ("PdS", i)) and oring.get(i % oslots) == i
-            if more:
+            yield wait("PR", i & 1, i)
+            if more:  # the next Sᵀ ahead of dV
                 yield wait("RD", i & 1, i)
                 yield wait(("QF", (i + 1) % qslots), ((i + 1) // qslots) & 1, (i + 1) // qslots)
                 issue_s(i + 1)
+            # dV from Pᵀ_i and dO_i
+            assert reg[i % 2] in (("P", i), ("PdS", i)) and oring.get(i % oslots) == i
             yield wait("DS", i & 1, i)  # dK from dSᵀ_i and Q_i
             assert reg[i % 2] == ("PdS", i) and qring.get(i % qslots) == i
             qring[i % qslots] = None
