@@ -22,7 +22,8 @@
 // Warp roles (384 threads, as in the forward): warps 0-3 and 4-7 do the
 // elementwise work of columns 0-63 and 64-127 of every row (one thread per
 // TMEM lane, so no row needs a reduction: D and the LSE are precomputed);
-// warp 8 issues the TMA loads; warp 9 allocates TMEM and issues the MMAs.
+// warp 8 issues the TMA loads; warp 9 allocates TMEM and issues the MMAs;
+// warp 10 issues the dP products (dQ kernel) or the dO loads (dK/dV kernel).
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -232,7 +233,7 @@ constexpr uint32_t kQBarQD = 0, kQBarKF = 1, kQBarKE = kQBarKF + kQKSlots,
                    kQBarVF = kQBarKE + kQKSlots, kQBarVE = kQBarVF + kQVSlots,
                    kQBarS = kQBarVE + kQVSlots, kQBarDP = kQBarS + 2, kQBarDS = kQBarDP + 1,
                    kQBarRD = kQBarDS + 2, kQBarDone = kQBarRD + 1, kQBarDrain = kQBarDone + 1,
-                   kQNumBars = kQBarDrain + 1;
+                   kQBarDrainP = kQBarDrain + 1, kQNumBars = kQBarDrainP + 1;
 // dS barriers alternate by step parity: the elementwise warps can finish step
 // j + 1 before the MMA thread has seen step j (the next dP starts on the
 // read-done signal), and a single barrier could then run two phases ahead
@@ -285,6 +286,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     mbar_init(bar(kQBarRD), 256);
     mbar_init(bar(kQBarDone), 1);
     mbar_init(bar(kQBarDrain), 1);
+    mbar_init(bar(kQBarDrainP), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -342,8 +344,12 @@ __global__ void __launch_bounds__(kBThreads, 1)
       for (int i = j - kQVSlots < 0 ? 0 : j - kQVSlots; i < j; ++i)
         wait_drain(bar(kQBarVF + i % kQVSlots), uint32_t(i / kQVSlots) & 1u);
       wait_drain(bar(kQBarQD), 0);
-    } else if (warp == 9) {
+    } else if (warp == 9 || warp == 10) {
       // ---------------------------------------------------------------- MMA
+      // Two issuing threads, so that neither product stream waits behind the
+      // other's barrier: warp 9 issues S = Q Kᵀ and dQ += dS K, warp 10 the
+      // dP = dO Vᵀ products (on disjoint TMEM columns and operands; each
+      // thread's commits track its own products).
       int n = 0;  // live key tiles of this query tile, counted by the warp
       for (int e0 = 0; e0 < len; e0 += 32) {
         const bool live = e0 + lane < len && cls_of(e0 + lane) != SCA_TILE_EMPTY;
@@ -361,57 +367,59 @@ __global__ void __launch_bounds__(kBThreads, 1)
           return wait_bar(bar(kQBarVF + j % kQVSlots), uint32_t(j / kQVSlots) & 1u, ctl, p.status,
                           p.timeout_ns);
         };
+        auto issue_dp = [&](int j) {  // dP_j = dO V_jᵀ; the last read of V_j
+          mma_qk8(tDP, dDO, desc_kmajor(vslot(j)), kIdescQK);
+          mma_commit(bar(kQBarDP));
+          mma_commit(bar(kQBarVE + j % kQVSlots));
+        };
         // Q and dO are always loaded: wait for them even with no key tile
         bool ok = wait_bar(bar(kQBarQD), 0, ctl, p.status, p.timeout_ns);
-        if (ok && n > 0) {
-          ok = wait_k(0);
-          if (ok) {
+        if (warp == 9) {
+          if (ok && n > 0 && (ok = wait_k(0))) {
             tc_fence_after();
             mma_qk8(tS0, dQ, desc_kmajor(kslot(0)), kIdescQK);
             mma_commit(bar(kQBarS));
-            ok = wait_v(0);
-          }
-          if (ok) {
-            tc_fence_after();
-            mma_qk8(tDP, dDO, desc_kmajor(vslot(0)), kIdescQK);
-            mma_commit(bar(kQBarDP));
-            mma_commit(bar(kQBarVE));
           }
           if (ok && n > 1 && (ok = wait_k(1))) {
             tc_fence_after();
             mma_qk8(tS0 + 128, dQ, desc_kmajor(kslot(1)), kIdescQK);
             mma_commit(bar(kQBarS + 1));
           }
-        }
-        for (int j = 0; ok && j < n; ++j) {
-          const uint32_t tSj = tS0 + uint32_t(j & 1) * 128;
+          for (int j = 0; ok && j < n; ++j) {
+            const uint32_t tSj = tS0 + uint32_t(j & 1) * 128;
+            if (!(ok = wait_bar(bar(kQBarDS + (j & 1)), uint32_t(j >> 1) & 1u, ctl, p.status,
+                                p.timeout_ns)))
+              break;
+            tc_fence_after();
+            mma_ts8_split(tDQ, tSj, tSj + 64, desc_mnmajor(kslot(j)), kIdescPV, j > 0 ? 1u : 0u);
+            mma_commit(bar(kQBarKE + j % kQKSlots));
+            if (j + 2 < n) {  // S of the key tile after next into the slot dS_j leaves
+              if (!(ok = wait_k(j + 2))) break;
+              tc_fence_after();
+              mma_qk8(tSj, dQ, desc_kmajor(kslot(j + 2)), kIdescQK);
+              mma_commit(bar(kQBarS + (j & 1)));
+            }
+          }
+          mma_commit(bar(kQBarDone));
+          mma_commit(bar(kQBarDrain));
+          wait_drain(bar(kQBarDrain), 0);
+        } else {
+          if (ok && n > 0 && (ok = wait_v(0))) {
+            tc_fence_after();
+            issue_dp(0);
+          }
           // dP of the next key tile as soon as dP_j has been read out: it
           // overlaps the elementwise work on this one
-          if (!(ok = wait_bar(bar(kQBarRD), uint32_t(j) & 1u, ctl, p.status, p.timeout_ns))) break;
-          tc_fence_after();
-          if (j + 1 < n) {
-            if (!(ok = wait_v(j + 1))) break;
+          for (int j = 0; ok && j + 1 < n; ++j) {
+            if (!(ok = wait_bar(bar(kQBarRD), uint32_t(j) & 1u, ctl, p.status, p.timeout_ns) &&
+                       wait_v(j + 1)))
+              break;
             tc_fence_after();
-            mma_qk8(tDP, dDO, desc_kmajor(vslot(j + 1)), kIdescQK);
-            mma_commit(bar(kQBarDP));
-            mma_commit(bar(kQBarVE + (j + 1) % kQVSlots));
+            issue_dp(j + 1);
           }
-          if (!(ok = wait_bar(bar(kQBarDS + (j & 1)), uint32_t(j >> 1) & 1u, ctl, p.status,
-                              p.timeout_ns)))
-            break;
-          tc_fence_after();
-          mma_ts8_split(tDQ, tSj, tSj + 64, desc_mnmajor(kslot(j)), kIdescPV, j > 0 ? 1u : 0u);
-          mma_commit(bar(kQBarKE + j % kQKSlots));
-          if (j + 2 < n) {  // S of the key tile after next into the slot dS_j leaves
-            if (!(ok = wait_k(j + 2))) break;
-            tc_fence_after();
-            mma_qk8(tSj, dQ, desc_kmajor(kslot(j + 2)), kIdescQK);
-            mma_commit(bar(kQBarS + (j & 1)));
-          }
+          mma_commit(bar(kQBarDrainP));
+          wait_drain(bar(kQBarDrainP), 0);
         }
-        mma_commit(bar(kQBarDone));
-        mma_commit(bar(kQBarDrain));
-        wait_drain(bar(kQBarDrain), 0);
       }
       __syncwarp();
     }

@@ -232,35 +232,21 @@ def backward_dq(n, seed, ks=3, vs=2):
             bars[("VF", j % vs)].expect(1)
             yield ("copy", ("VF", j % vs), 1)
 
-    def mma():
+    def qk(j, buf):
+        assert kslot[j % ks] == j and sbuf.get(buf) in (None, "read")
+        sbuf[buf] = ("S", j)
+
+    def mma_s_dq():  # one issuing thread: S = Q Kᵀ and dQ += dS K
         yield wait("QD", 0, 0)
-
-        def qk(j, buf):
-            assert kslot[j % ks] == j and sbuf.get(buf) in (None, "read")
-            sbuf[buf] = ("S", j)
-
         if n:
             yield wait(("KF", 0), 0, 0)
             qk(0, 0)
             bars[("S", 0)].arrive()
-            yield wait(("VF", 0), 0, 0)
-            dp["v"] = 0
-            bars["DP"].arrive()
-            vslot[0] = None
-            bars[("VE", 0)].arrive()
-            if n > 1:
-                yield wait(("KF", 1), 0, 0)
-                qk(1, 1)
-                bars[("S", 1)].arrive()
+        if n > 1:
+            yield wait(("KF", 1), 0, 0)
+            qk(1, 1)
+            bars[("S", 1)].arrive()
         for j in range(n):
-            yield wait("RD", j & 1, j)
-            if j + 1 < n:
-                yield wait(("VF", (j + 1) % vs), ((j + 1) // vs) & 1, (j + 1) // vs)
-                assert vslot[(j + 1) % vs] == j + 1 and dp.get("read") == j
-                dp["v"] = j + 1
-                bars["DP"].arrive()
-                vslot[(j + 1) % vs] = None
-                bars[("VE", (j + 1) % vs)].arrive()
             yield wait(("DS", j & 1), (j >> 1) & 1, j >> 1)
             assert sbuf[j & 1] == ("dS", j) and kslot[j % ks] == j
             sbuf[j & 1] = "read"
@@ -271,6 +257,23 @@ def backward_dq(n, seed, ks=3, vs=2):
                 qk(j + 2, j & 1)
                 bars[("S", j & 1)].arrive()
         bars["DONE"].arrive()
+
+    def issue_dp(j):
+        assert vslot[j % vs] == j and (j == 0 or dp.get("read") == j - 1)
+        dp["v"] = j
+        bars["DP"].arrive()
+        vslot[j % vs] = None
+        bars[("VE", j % vs)].arrive()
+
+    def mma_dp():  # the other issuing thread: dP = dO Vᵀ
+        yield wait("QD", 0, 0)
+        if n:
+            yield wait(("VF", 0), 0, 0)
+            issue_dp(0)
+        for j in range(n - 1):
+            yield wait("RD", j & 1, j)
+            yield wait(("VF", (j + 1) % vs), ((j + 1) // vs) & 1, (j + 1) // vs)
+            issue_dp(j + 1)
 
     def elementwise():
         for j in range(n):
@@ -284,7 +287,8 @@ def backward_dq(n, seed, ks=3, vs=2):
             bars[("DS", j & 1)].arrive()
         yield wait("DONE", 0, 0)
 
-    run({"producer": producer(), "mma": mma(), "elementwise": elementwise()}, bars, seed)
+    run({"producer": producer(), "mma_s_dq": mma_s_dq(), "mma_dp": mma_dp(),
+         "elementwise": elementwise()}, bars, seed)
 
 
 def backward_dkdv(n, seed, qslots=3, oslots=2):
