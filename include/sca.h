@@ -391,7 +391,10 @@ SCA_API int sca_action_causal_attn_fwd_static_ws(const sca_kv_cache* cache,
  * Three kernels on the stream: D and LSE, dQ (query tiles over their key
  * tiles), dK and dV (key tiles over the query tiles that see them); no
  * atomics, so the result does not depend on scheduling. The call allocates
- * nothing. A key no query sees gets dK = dV = 0. */
+ * nothing. A key no query sees gets dK = dV = 0. The dK/dV kernel uses all
+ * 227 KB of shared memory a CTA may have and needs its dynamic shared memory
+ * to start on a 1024-byte boundary (as on B200); if it does not, the kernel
+ * does nothing and writes SCA_ERR_MISALIGNED to dev_status. */
 SCA_API int sca_action_causal_attn_bwd(const sca_metadata* md, int32_t heads, const void* q,
                                        const void* k, const void* v, const void* o,
                                        const float* lse, const void* d_o, void* dq, void* dk,
