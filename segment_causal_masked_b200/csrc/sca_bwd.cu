@@ -703,20 +703,19 @@ __global__ void __launch_bounds__(kBThreads, 1)
         // dV += Pᵀ_i dO_i (B MN-major: rows are queries)
         tc_fence_after();
         mma_ts8_blocks(tDV, region(i), desc_mnmajor(oslot(i)), kIdescPV, i > 0 ? 1u : 0u);
-        // dK += dSᵀ_i Q_i
-        if (!(ok = wait_bar(bar(kKBarDS), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns))) break;
+        // dK += dSᵀ_i Q_i, then dPᵀ_{i+1} into region(i) right behind it (the
+        // next dO stage is waited for first, so the two go out back to back;
+        // the in-order pipe runs dPᵀ after dV and dK have read the region)
+        if (!(ok = (!more || wait_o(i + 1)) &&
+                   wait_bar(bar(kKBarDS), uint32_t(i) & 1u, ctl, p.status, p.timeout_ns)))
+          break;
         tc_fence_after();
         mma_ts8_blocks(tDK, region(i) + 64, desc_mnmajor(qslot(i)), kIdescPV, i > 0 ? 1u : 0u);
         mma_commit(bar(kKBarQE + i % kKQSlots));  // the last read of Q_i
         // the dO stage too: dV has read dO_i and the elementwise warps their
         // −D and −L before arriving on dSᵀ
         mma_commit(bar(kKBarOE + i % kKOSlots));
-        // dPᵀ_{i+1} into region(i), after dV and dK have read it (in-order pipe)
-        if (more) {
-          if (!(ok = wait_o(i + 1))) break;
-          tc_fence_after();
-          issue_dp(i + 1);
-        }
+        if (more) issue_dp(i + 1);
       }
       mma_commit(bar(kKBarDone));
       mma_commit(bar(kKBarDrain));

@@ -359,6 +359,8 @@ def backward_dkdv(n, seed, qslots=3, oslots=2):
                 issue_s(i + 1)
             # dV from Pᵀ_i and dO_i
             assert reg[i % 2] in (("P", i), ("PdS", i)) and oring.get(i % oslots) == i
+            if more:  # the next dO stage first, so that dK and the next dPᵀ go out together
+                yield wait(("OF", (i + 1) % oslots), ((i + 1) // oslots) & 1, (i + 1) // oslots)
             yield wait("DS", i & 1, i)  # dK from dSᵀ_i and Q_i
             assert reg[i % 2] == ("PdS", i) and qring.get(i % qslots) == i
             qring[i % qslots] = None
@@ -366,7 +368,6 @@ def backward_dkdv(n, seed, qslots=3, oslots=2):
             oring[i % oslots] = None  # dV and the elementwise warps are done with the dO stage
             bars[("OE", i % oslots)].arrive()
             if more:
-                yield wait(("OF", (i + 1) % oslots), ((i + 1) // oslots) & 1, (i + 1) // oslots)
                 issue_dp(i + 1)
         bars["DONE"].arrive()
 
