@@ -14,20 +14,24 @@ The oracle is written from the pages' prose, in plain NumPy, in float64:
 * ``schedule``  - brute-force 128x128 tile classification from the explicit
                   mask, and the unmasked-pair count A of Eq. 6;
 * ``cache``     - the growing KV cache after an append, and the descriptor
-                  words the library's ABI documents.
+                  words the library's ABI documents;
+* ``camera``    - the camera cross-attention of Eq. 3 on projected inputs
+                  (visual queries over one segment's camera tokens).
 
 Pages cited (title, section):
 
 * [picx]   "Hy-Nomas" technical-report summary on picx.dev: Methodology >
            Model Architecture ("Segment-wise Causal Attention",
-           "Action-Aware Causal Attention (Figure 6b)"); Training
+           "Action-Aware Causal Attention (Figure 6b)", "Camera-Trajectory
+           Conditioning", Eq. 3); Training
            Infrastructure (Eq. 6, "Flex-Flash-Attention").
 * [gpts24] "Tencent's Hy-Nomas Steers a 60-Second Video World With Text and
            Camera on One RTX 4090": "One World, Generated Segment by
            Segment" (the growing KV cache); "Inside the Architecture"
            (action-aware causal attention).
 * [onedev] onedev.kr review "Hy-Nomas가 8B 모델 하나로 ...": "무엇과 다른가"
-           (the head/tail split and who may see what).
+           (the head/tail split and who may see what); "어떻게 쓰나" (one
+           camera token per latent frame, time-aligned cross-attention).
 * [xyznot] "Hy-Nomas: Serbest Biçimli Etkileşimli Dünya Üretimine Doğru":
            "Eyleme Duyarlı Nedensel Dikkat ve Kamera Koşullandırması";
            "Dağıtık Paketleme FLOP Tahmini" (A_i of Eq. 6).
