@@ -72,18 +72,28 @@ BWD_WORKLOADS = {"packed-360k-bwd", "packed-64k-bwd"}
 WORKLOADS["480p-single-turn-4nfe"] = lambda: dataclasses.replace(
     W.session_480p_single_turn(), name="480p-single-turn-4nfe")
 NFE_WORKLOADS = {"480p-single-turn-4nfe": 4}
+# the camera cross-attention of one 480p segment (out = x + softmax(q k_camᵀ)
+# v_cam): an HBM-bound call with its own metric, GB/s of algorithmic bytes
+WORKLOADS["camera-xattn-480p"] = W.camera_480p
+CAMERA_WORKLOADS = {"camera-xattn-480p"}
+CAMERA_METRIC = "camera cross-attention HBM GB/s (algorithmic bytes) and % of measured copy bandwidth"
+CAMERA_INPUT_SETS = 4   # (q, x, out) sets rotated over the steps: 4 x 149 MB > L2
 # a timed call this long runs at the power-capped clock: its fraction is taken
 # against the sustained bf16 peak, shorter calls against the burst peak
 SUSTAINED_CALL_MS = 500.0
 BWD_FLOP_FACTOR = 2.5   # five products per visible pair against the forward's two
-KERNEL_SOURCES = ["segment_causal_masked_b200/csrc/sca_kernels.cu",
-                  "segment_causal_masked_b200/csrc/sca_ptx.cuh",
-                  "segment_causal_masked_b200/csrc/sca_internal.h"]
+KERNEL_SOURCES = {
+    "attn_fwd_kernel": ["segment_causal_masked_b200/csrc/sca_kernels.cu",
+                        "segment_causal_masked_b200/csrc/sca_ptx.cuh",
+                        "segment_causal_masked_b200/csrc/sca_internal.h"],
+    "camera_xattn_kernel": ["segment_causal_masked_b200/csrc/sca_camera.cu",
+                            "segment_causal_masked_b200/csrc/sca_camera.h"],
+}
 
 
-def kernel_hash() -> str:
+def kernel_hash(kernel: str = "attn_fwd_kernel") -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -111,7 +121,7 @@ def stored_traffic(kernel: str, workload: str):
     with open(path) as f:
         d = json.load(f)
     e = d.get(kernel, {}).get(workload)
-    if not e or e.get("kernel_hash") != kernel_hash():
+    if not e or e.get("kernel_hash") != kernel_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -230,6 +240,48 @@ class OracleSample:
         return time.perf_counter() - t0
 
 
+def camera_bytes(cp) -> int:
+    """Algorithmic HBM bytes of one camera cross-attention call: q and x read
+    and out written (bf16 [n_q, heads, 128]), the camera K and V read once,
+    and the int32 frame index of every query in the frame-aligned modes."""
+    row = cp.n_q * cp.heads * W.HEAD_DIM * 2
+    return 3 * row + 2 * cp.n_cam * cp.heads * W.HEAD_DIM * 2 + (4 * cp.n_q if cp.mode else 0)
+
+
+class CameraOracleSample:
+    """The camera oracle on `rows` query rows of the workload (every head),
+    inputs drawn once; throughput counted in the same algorithmic bytes per
+    row as the kernel's."""
+
+    def __init__(self, cp, rows: int, seed: int = 9):
+        import numpy as np
+        import torch
+
+        torch.set_num_threads(os.cpu_count() or 1)
+        self.cp = cp
+        rows = min(rows, cp.n_q)
+        self.rows = np.linspace(0, cp.n_q - 1, rows).round().astype(np.int64)
+        shp = (rows, cp.heads, W.HEAD_DIM)
+        self.q = W.randn_bf16(shp, 1000 * seed).float().numpy()
+        self.x = W.randn_bf16(shp, 1000 * seed + 1).float().numpy()
+        cam = (cp.n_cam, cp.heads, W.HEAD_DIM)
+        self.k = W.randn_bf16(cam, 1000 * seed + 2).float().numpy()
+        self.v = W.randn_bf16(cam, 1000 * seed + 3).float().numpy()
+        self.frame = cp.q_frame()[self.rows]
+        self.bytes = camera_bytes(cp) * rows / cp.n_q
+        self.desc = (f"oracle (float64 NumPy) on {rows} of the {cp.n_q} query rows x "
+                     f"{cp.heads} heads of {cp.name}, as GB/s of the kernel's algorithmic "
+                     f"bytes for those rows")
+
+    def run(self) -> float:
+        from oracle import camera as ocam
+
+        t0 = time.perf_counter()
+        ocam.camera_cross_attention(self.q, self.k, self.v, self.x, self.frame, self.cp.mode,
+                                    self.cp.softmax_scale)
+        return time.perf_counter() - t0
+
+
 def cpu_model() -> str:
     """The host CPU's model name (first 'model name' of /proc/cpuinfo)."""
     try:
@@ -258,26 +310,36 @@ def run_reference(args, problem):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    bwd = args.workload in BWD_WORKLOADS
-    sample = OracleSample(problem, args.oracle_rows // (8 if bwd else 1),
-                          int8=args.workload in INT8_WORKLOADS, backward=bwd)
+    if args.workload in CAMERA_WORKLOADS:
+        sample = CameraOracleSample(problem, problem.n_q)   # the whole call
+        metric, unit = CAMERA_METRIC, "GB/s"
+        units = lambda sec: sample.bytes / sec / 1e9  # noqa: E731
+        config = {"workload": problem.name, "queries": problem.n_q,
+                  "camera_tokens": problem.n_cam, "heads": problem.heads,
+                  "head_dim": W.HEAD_DIM, "mode": problem.mode}
+    else:
+        bwd = args.workload in BWD_WORKLOADS
+        sample = OracleSample(problem, args.oracle_rows // (8 if bwd else 1),
+                              int8=args.workload in INT8_WORKLOADS, backward=bwd)
+        metric, unit = METRIC, "TFLOP/s"
+        units = lambda sec: sample.flops / sec / 1e12  # noqa: E731
+        config = {"workload": problem.name, "queries": problem.n_query_tokens,
+                  "keys": problem.n_key_tokens, "heads": problem.heads, "head_dim": W.HEAD_DIM}
     for _ in range(args.warmup):
         sample.run()
     secs = [sample.run() for _ in range(args.steps)]
-    vals = [sample.flops / s / 1e12 for s in secs]
+    vals = [units(s) for s in secs]
     desc = sample.desc
-    rows_per_step = len(sample.rows)
+    config["sample_rows_per_step"] = len(sample.rows)
     value = statistics.mean(vals)
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": unit,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * statistics.mean(secs), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": problem.name, "queries": problem.n_query_tokens,
-                       "keys": problem.n_key_tokens, "heads": problem.heads,
-                       "head_dim": W.HEAD_DIM, "sample_rows_per_step": rows_per_step},
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cpu_threads(),
+            "config": config,
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cpu_threads(),
                              "cpu_model": cpu_model(), "kind": "oracle", "sample": desc},
-            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -425,7 +487,10 @@ class Session:
             self.cache.truncate(self.n_prior)
 
 
-def run_native(args, problem):
+def init_ranks(args):
+    """(world, rank, local rank) from the torchrun environment; the device
+    set and, for N > 1, the NCCL process group up (used for the barrier and
+    the max over ranks only)."""
     import torch
     import torch.distributed as dist
 
@@ -439,6 +504,14 @@ def run_native(args, problem):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def run_native(args, problem):
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = init_ranks(args)
 
     def barrier():
         if world > 1:
@@ -628,6 +701,160 @@ def run_native(args, problem):
     return 0
 
 
+def run_camera(args, cp):
+    """The camera cross-attention call of one segment, timed per call on the
+    device (inputs rotated over CAMERA_INPUT_SETS sets larger than L2 together)
+    and end to end with its inputs uploaded from and its output read back to
+    pinned host memory every step."""
+    import torch
+    import torch.distributed as dist
+
+    from segment_causal_masked_b200 import sca
+
+    world, rank, local = init_ranks(args)
+    dev = torch.device("cuda", local)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 * 5 + rank)
+    bf = torch.bfloat16
+    shp, cam = (cp.n_q, cp.heads, W.HEAD_DIM), (cp.n_cam, cp.heads, W.HEAD_DIM)
+    sets = [[torch.randn(shp, generator=g, device=dev).to(bf) for _ in range(3)]
+            for _ in range(CAMERA_INPUT_SETS)]   # q, x, out
+    k_cam = torch.randn(cam, generator=g, device=dev).to(bf)
+    v_cam = torch.randn(cam, generator=g, device=dev).to(bf)
+    frame = torch.from_numpy(cp.q_frame()).to(dev)
+    stream = torch.cuda.current_stream()
+
+    def call(q, x, out, fr, kc, vc):
+        sca.camera_cross_attn(q, kc, vc, x, out, fr, cp.mode, cp.softmax_scale,
+                              stream.cuda_stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        q, x, out = sets[i % CAMERA_INPUT_SETS]
+        call(q, x, out, frame, k_cam, v_cam)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record(stream)
+    for i in range(args.steps):
+        q, x, out = sets[i % CAMERA_INPUT_SETS]
+        evs[i][0].record(stream)
+        call(q, x, out, frame, k_cam, v_cam)
+        evs[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clock_info = clocks.stop()
+    barrier()
+    nbytes = camera_bytes(cp)
+    ms_total = reduce_max(t0.elapsed_time(t1), world, "cuda")
+    call_ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in evs), world, "cuda")
+    value = world * nbytes * args.steps / (ms_total * 1e-3) / 1e9
+
+    # end to end: q, x, the frames and the camera K/V uploaded from pinned
+    # host memory, the call, out read back; uploads of step i+1 (one stream)
+    # and the read-back of step i (another) overlap step i's call
+    host_in = [t.cpu().pin_memory() for t in (sets[0][0], sets[0][1], frame, k_cam, v_cam)]
+    host_out = torch.empty(shp, dtype=bf, pin_memory=True)
+    dev_in = [[torch.empty_like(t, device=dev) for t in host_in] for _ in range(2)]
+    dev_out = [torch.empty(shp, dtype=bf, device=dev) for _ in range(2)]
+    bytes_in = sum(t.numel() * t.element_size() for t in host_in)
+    bytes_out = host_out.numel() * host_out.element_size()
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = torch.cuda.Event
+    in_ready, out_ready, out_read = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    used = [None, None]
+
+    def upload(i):
+        b = i % 2
+        with torch.cuda.stream(h2d):
+            if used[b] is not None:
+                h2d.wait_event(used[b])
+            for dst, src in zip(dev_in[b], host_in):
+                dst.copy_(src, non_blocking=True)
+            in_ready[b].record(h2d)
+
+    def e2e_steps(n):
+        upload(0)
+        for i in range(n):
+            b = i % 2
+            if i + 1 < n:
+                upload(i + 1)
+            stream.wait_event(in_ready[b])
+            stream.wait_event(out_read[b])
+            q, x, fr, kc, vc = dev_in[b]
+            call(q, x, dev_out[b], fr, kc, vc)
+            used[b] = ev()
+            used[b].record(stream)
+            out_ready[b].record(stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(out_ready[b])
+                host_out.copy_(dev_out[b], non_blocking=True)
+                out_read[b].record(d2h)
+        last = ev()
+        last.record(d2h)
+        stream.wait_event(last)
+
+    e2e_steps(args.warmup)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(stream)
+    h2d.wait_event(e0)
+    e2e_steps(args.steps)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = reduce_max(e0.elapsed_time(e1), world, "cuda")
+    e2e_value = world * nbytes * args.steps / (e2e_ms * 1e-3) / 1e9
+
+    if rank == 0:
+        peaks = measured_peaks()
+        peak = float(peaks["hbm_gbs"])
+        achieved = nbytes / (call_ms * 1e-3) / 1e9
+        traffic = stored_traffic("camera_xattn_kernel", cp.name)
+        line = {
+            "metric": CAMERA_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": cp.name, "queries": cp.n_q, "camera_tokens": cp.n_cam,
+                       "heads": cp.heads, "head_dim": W.HEAD_DIM, "mode": cp.mode,
+                       "algorithmic_bytes_per_step": nbytes,
+                       "step": "one camera cross-attention call (out = x + attention)",
+                       "l2": "q, x, out rotated over %d sets (%.0f MB together) > L2"
+                             % (CAMERA_INPUT_SETS, CAMERA_INPUT_SETS * 3 * cp.n_q * cp.heads
+                                * W.HEAD_DIM * 2 / 1e6),
+                       "parallelism": f"replicas x{world}"},
+            "pct_of_peak": 100.0 * value / world / peak,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "camera_xattn_kernel", "kernel_ms": call_ms,
+                         "peak_source": f"{peaks['source']} HBM copy bandwidth"},
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": bytes_in,
+                    "d2h_bytes_per_step": bytes_out, "ms_per_step": e2e_ms / args.steps},
+            "gpu_launches": args.steps,
+            "clocks": clock_info,
+        }
+        if not args.no_cpu_baseline:
+            sample = CameraOracleSample(cp, cp.n_q)   # the whole call
+            dt = sample.run()
+            line["cpu_baseline"] = {"value": sample.bytes / dt / 1e9, "unit": "GB/s",
+                                    "cores": cpu_threads(), "cpu_model": cpu_model(),
+                                    "kind": "oracle", "sample": sample.desc, "seconds": dt}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -645,6 +872,8 @@ def main():
     problem = WORKLOADS[args.workload]()
     if args.impl == "reference":
         return run_reference(args, problem)
+    if args.workload in CAMERA_WORKLOADS:
+        return run_camera(args, problem)
     return run_native(args, problem)
 
 

@@ -415,6 +415,43 @@ SCA_API int sca_metadata_get_bwd_schedule(const sca_metadata* md, const int32_t*
 /* Workspace the backward needs: 2 · heads · round_up(n, 128) floats. */
 SCA_API int sca_attn_bwd_workspace_bytes(const sca_metadata* md, int32_t heads, uint64_t* bytes);
 
+/* ---------------------------------------------------------------------------
+ * Camera cross-attention of one segment: the attention core of Eq. 3 of
+ * [picx.dev summary, Methodology › Model Architecture, Camera-Trajectory
+ * Conditioning], V~ = V + CrossAttn(V, C), with the visual tokens as queries
+ * and the segment's camera tokens (one per latent frame, aligned in time with
+ * the frames [onedev.kr review, "어떻게 쓰나"]) as keys and values, on inputs
+ * already projected per head (the projections are model weights):
+ *
+ *   out_i = x_i + sum_f softmax_f(softmax_scale · <q_i, k_f>) v_f
+ *
+ * over the camera tokens f that query i sees. The pages leave that set open
+ * beyond "time-aligned"; `mode` picks a reading:
+ *   SCA_CAM_ALL         every camera token of the segment;
+ *   SCA_CAM_OWN_FRAME   only the token of the query's own latent frame;
+ *   SCA_CAM_UP_TO_FRAME the tokens of latent frames 0 .. the query's own.
+ * A query whose frame lies outside [0, n_cam) sees no token in the two
+ * frame modes and keeps out_i = x_i.
+ * Arguments:
+ *   q, x, out : bf16 token-major [n_q][heads][128] (16-byte aligned); out
+ *            may be x (the residual updated in place), no other overlap;
+ *   q_frame : int32 [n_q], each query's latent frame in the segment; may be
+ *            NULL for SCA_CAM_ALL;
+ *   k_cam, v_cam : bf16 [n_cam][heads][128] (16-byte aligned);
+ *   n_q >= 0, 1 <= n_cam <= SCA_MAX_CAMERA_TOKENS, heads >= 1;
+ *   softmax_scale : finite (1/sqrt(128) for the model's heads).
+ * S and O are accumulated in fp32, P is rounded to bf16 for its product, the
+ * output is rounded once to bf16. Enqueued on `stream`; allocates nothing.
+ * SCA_ERR_INVALID_ARG / SCA_ERR_MISALIGNED on bad arguments, and
+ * SCA_ERR_UNSUPPORTED past 65,535 heads or 2^31 elements of q (nothing is
+ * launched then). */
+enum { SCA_CAM_ALL = 0, SCA_CAM_OWN_FRAME = 1, SCA_CAM_UP_TO_FRAME = 2 };
+#define SCA_MAX_CAMERA_TOKENS 64
+SCA_API int sca_camera_cross_attn(const void* q, const int32_t* q_frame, const void* k_cam,
+                                  const void* v_cam, const void* x, void* out, int32_t n_q,
+                                  int32_t n_cam, int32_t heads, int32_t mode,
+                                  float softmax_scale, void* stream);
+
 /* Message of the calling thread's last failure ("" if none). */
 SCA_API const char* sca_last_error(void);
 

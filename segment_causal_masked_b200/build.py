@@ -19,8 +19,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsca.so")
-SOURCES = ["sca_host.cpp", "sca_kernels.cu", "sca_bwd.cu", "sca_static_ws.cu"]
-HEADERS = ["sca_internal.h", "sca_ptx.cuh"]
+SOURCES = ["sca_host.cpp", "sca_kernels.cu", "sca_bwd.cu", "sca_static_ws.cu", "sca_camera.cu"]
+HEADERS = ["sca_internal.h", "sca_ptx.cuh", "sca_camera.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 # Registers per thread that each warp-specialised kernel must be launched
 # with: its setmaxnreg split (static_asserts beside the kernels) adds up to

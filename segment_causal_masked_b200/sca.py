@@ -26,6 +26,8 @@ TILE = 128
 MAX_ACTIONS = 32
 TEXTQ_OWN_TAIL, TEXTQ_FULL_SEGMENT = 0, 1
 TILE_EMPTY, TILE_PARTIAL, TILE_FULL = 0, 1, 2
+CAM_ALL, CAM_OWN_FRAME, CAM_UP_TO_FRAME = 0, 1, 2
+MAX_CAMERA_TOKENS = 64
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_MISALIGNED = 0, -1, -2, -3
 ERR_CAPACITY, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_MISMATCH = -4, -5, -6, -7
 
@@ -40,7 +42,7 @@ EXPORTED = (
     "sca_action_causal_attn_fwd", "sca_action_causal_attn_fwd_static_ws",
     "sca_attn_workspace_bytes", "sca_attn_plan", "sca_attn_plan_for_sms",
     "sca_attn_int8_scratch_bytes",
-    "sca_action_causal_attn_bwd", "sca_attn_bwd_workspace_bytes",
+    "sca_action_causal_attn_bwd", "sca_attn_bwd_workspace_bytes", "sca_camera_cross_attn",
     "sca_set_split_override", "sca_set_pipeline_timeout_ns",
     "sca_last_error", "sca_read_device_status", "sca_debug_bounded_wait",
 )
@@ -100,6 +102,7 @@ _SIGS = {
     "sca_action_causal_attn_bwd": [_P, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_float,
                                    _P, ctypes.c_uint64, _P, _P],
     "sca_attn_bwd_workspace_bytes": [_P, _i32, ctypes.POINTER(ctypes.c_uint64)],
+    "sca_camera_cross_attn": [_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, ctypes.c_float, _P],
     "sca_attn_plan": [_P, _i32, _pi32, _pi32, _pi32],
     "sca_attn_plan_for_sms": [_P, _i32, _i32, _pi32, _pi32, _pi32, ctypes.POINTER(ctypes.c_uint64)],
     "sca_set_split_override": [_i32],
@@ -400,6 +403,22 @@ def action_causal_attn_bwd(md: Metadata, heads: int, q, k, v, o, lse, d_o, dq, d
                                            _ptr(dv), float(softmax_scale), _ptr(workspace),
                                            int(workspace_bytes or 0), _ptr(dev_status),
                                            _stream(stream)))
+
+
+def camera_cross_attn(q, k_cam, v_cam, x, out, q_frame=None, mode: int = CAM_ALL,
+                      softmax_scale: float = 128 ** -0.5, stream=None) -> None:
+    """out = x + the camera cross-attention of queries ``q`` over one
+    segment's camera tokens (see include/sca.h). ``q``, ``x``, ``out``: bf16
+    [n_q, heads, 128] (``out`` may be ``x``); ``k_cam``, ``v_cam``: bf16
+    [n_cam, heads, 128]; ``q_frame``: int32 [n_q] or None (SCA_CAM_ALL)."""
+    n_q, heads = int(q.shape[0]), int(q.shape[1])
+    if tuple(x.shape) != tuple(q.shape) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q, x and out must have the same shape [n_q, heads, 128]")
+    if tuple(v_cam.shape) != tuple(k_cam.shape) or tuple(k_cam.shape[1:]) != (heads, HEAD_DIM):
+        raise ValueError("k_cam and v_cam must be [n_cam, heads, 128]")
+    _check(_lib.sca_camera_cross_attn(_ptr(q), _ptr(q_frame), _ptr(k_cam), _ptr(v_cam), _ptr(x),
+                                      _ptr(out), n_q, int(k_cam.shape[0]), heads, int(mode),
+                                      float(softmax_scale), _stream(stream)))
 
 
 def attn_int8_scratch_bytes(md: Metadata, heads: int) -> int:

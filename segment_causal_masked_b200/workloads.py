@@ -121,6 +121,41 @@ def session_480p_long() -> Problem:
     return Problem("480p-long-session", (s,) * 12, (s,), heads=16)
 
 
+@dataclasses.dataclass(frozen=True)
+class CameraProblem:
+    """One camera cross-attention call: the video tokens of one segment
+    (frame-major, ``tokens_per_frame`` per latent frame) as queries over the
+    segment's camera tokens, one per latent frame ([onedev] "어떻게 쓰나")."""
+
+    name: str
+    num_frames: int
+    tokens_per_frame: int
+    heads: int = 16
+    mode: int = 0                       # 0 every token, 1 own frame, 2 frames up to its own
+
+    @property
+    def n_q(self) -> int:
+        return self.num_frames * self.tokens_per_frame
+
+    @property
+    def n_cam(self) -> int:
+        return self.num_frames
+
+    @property
+    def softmax_scale(self) -> float:
+        return 1.0 / math.sqrt(HEAD_DIM)
+
+    def q_frame(self) -> np.ndarray:
+        """int32 [n_q]: the latent frame of every query token."""
+        return (np.arange(self.n_q) // self.tokens_per_frame).astype(np.int32)
+
+
+def camera_480p(mode: int = 0) -> CameraProblem:
+    """The 12,090 video tokens of a 480p segment (31 latent frames of 15 x 26)
+    over its 31 camera tokens, 16 heads."""
+    return CameraProblem("camera-xattn-480p", 31, 15 * 26, 16, mode)
+
+
 def _windows_720p(rng: np.random.Generator, num_frames: int = 16,
                   n_actions: int = 6) -> Tuple[Tuple[int, int], ...]:
     """Random contiguous windows; redrawn until at least two overlap and at

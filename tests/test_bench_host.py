@@ -47,9 +47,9 @@ def test_stored_traffic_needs_the_current_kernel_source(tmp_path, monkeypatch):
     rec = {"attn_fwd_kernel": {"w": {"kernel_hash": "0" * 16, "dram_bytes_per_launch": 5}}}
     (prof / "traffic.json").write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "kernel_hash", lambda: "0" * 16)
+    monkeypatch.setattr(bench, "kernel_hash", lambda k: "0" * 16)
     assert bench.stored_traffic("attn_fwd_kernel", "w") == 5
-    monkeypatch.setattr(bench, "kernel_hash", lambda: "1" * 16)   # the kernel changed since
+    monkeypatch.setattr(bench, "kernel_hash", lambda k: "1" * 16)   # the kernel changed since
     assert bench.stored_traffic("attn_fwd_kernel", "w") is None
 
 

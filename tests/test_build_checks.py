@@ -120,13 +120,15 @@ def test_binding_constants_match_the_header():
         "SCA_ERR_DEVICE_TIMEOUT": sca.ERR_DEVICE_TIMEOUT, "SCA_ERR_MISMATCH": sca.ERR_MISMATCH,
         "SCA_TEXTQ_OWN_TAIL": sca.TEXTQ_OWN_TAIL, "SCA_TEXTQ_FULL_SEGMENT": sca.TEXTQ_FULL_SEGMENT,
         "SCA_TILE_EMPTY": sca.TILE_EMPTY, "SCA_TILE_PARTIAL": sca.TILE_PARTIAL,
-        "SCA_TILE_FULL": sca.TILE_FULL,
+        "SCA_TILE_FULL": sca.TILE_FULL, "SCA_CAM_ALL": sca.CAM_ALL,
+        "SCA_CAM_OWN_FRAME": sca.CAM_OWN_FRAME, "SCA_CAM_UP_TO_FRAME": sca.CAM_UP_TO_FRAME,
     }
     for name, value in pairs.items():
         assert enums[name] == value, name
     assert int(defines["SCA_HEAD_DIM"]) == sca.HEAD_DIM
     assert int(defines["SCA_TILE"]) == sca.TILE
     assert int(defines["SCA_MAX_ACTIONS"]) == sca.MAX_ACTIONS
+    assert int(defines["SCA_MAX_CAMERA_TOKENS"]) == sca.MAX_CAMERA_TOKENS
     m = re.match(r"\((\d+)ull\s*<<\s*(\d+)\)", defines["SCA_STATIC_WORKSPACE_BYTES"].strip())
     assert m and int(m.group(1)) << int(m.group(2)) == sca.STATIC_WORKSPACE_BYTES
 

@@ -1,0 +1,118 @@
+"""GPU parity of the camera cross-attention (sca_camera_cross_attn) against the
+oracle (Eq. 3 of [picx] "Camera-Trajectory Conditioning"; one camera token
+per latent frame, [onedev] "어떻게 쓰나").
+
+Bar: every output element within 1e-2 · max(1, |ref|) of the float64 oracle
+on the same bf16 inputs, and a relative L2 error <= 5e-3 (derived: P is
+rounded to bf16 before its product, 2^-9 relative, and the output is one
+bf16 rounding, 2^-9 relative, of x + the attention). Where a query sees a
+single camera token its weight is exactly 1 and the output is the bf16
+rounding of x + v, which the test checks bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import camera as ocam
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from segment_causal_masked_b200 import sca  # noqa: E402
+
+D = 128
+SCALE = D ** -0.5
+
+
+def _inputs(n_q, n_cam, heads, seed, sharp=1.0):
+    g = torch.Generator().manual_seed(seed)
+    q = (torch.randn(n_q, heads, D, generator=g) * sharp).bfloat16()
+    k = torch.randn(n_cam, heads, D, generator=g).bfloat16()
+    v = torch.randn(n_cam, heads, D, generator=g).bfloat16()
+    x = torch.randn(n_q, heads, D, generator=g).bfloat16()
+    frame = torch.randint(0, n_cam, (n_q,), generator=g, dtype=torch.int32)
+    return q, k, v, x, frame
+
+
+def _run(q, k, v, x, frame, mode, out=None):
+    qd, kd, vd, xd, fd = (t.cuda() for t in (q, k, v, x, frame))
+    od = torch.empty_like(xd) if out is None else out
+    sca.camera_cross_attn(qd, kd, vd, xd, od, fd, mode, SCALE)
+    torch.cuda.synchronize()
+    return od.cpu()
+
+
+def _ref(q, k, v, x, frame, mode):
+    return ocam.camera_cross_attention(q.float().numpy(), k.float().numpy(), v.float().numpy(),
+                                       x.float().numpy(), frame.numpy(), mode, SCALE)
+
+
+def _check(out, ref):
+    o = out.float().numpy().astype(np.float64)
+    d = np.abs(o - ref)
+    assert (d <= 1e-2 * np.maximum(1.0, np.abs(ref))).all(), f"max |d| = {d.max()}"
+    assert np.linalg.norm(o - ref) <= 5e-3 * np.linalg.norm(ref)
+
+
+@pytest.mark.parametrize("mode", [sca.CAM_ALL, sca.CAM_OWN_FRAME, sca.CAM_UP_TO_FRAME])
+@pytest.mark.parametrize("n_cam", [1, 5, 16, 31, 48, 64])
+def test_matches_oracle(mode, n_cam):
+    q, k, v, x, frame = _inputs(301, n_cam, 3, 100 + n_cam + 7 * mode)
+    _check(_run(q, k, v, x, frame, mode), _ref(q, k, v, x, frame, mode))
+
+
+@pytest.mark.parametrize("n_q", [1, 15, 16, 17, 2048])
+@pytest.mark.parametrize("sharp", [1.0, 8.0])
+def test_ragged_rows_and_sharp_scores(n_q, sharp):
+    q, k, v, x, frame = _inputs(n_q, 31, 16, 200 + n_q, sharp)
+    _check(_run(q, k, v, x, frame, sca.CAM_ALL), _ref(q, k, v, x, frame, sca.CAM_ALL))
+
+
+def test_own_frame_is_exact():
+    """One visible token: out = bf16(x + v[frame]) bit for bit."""
+    q, k, v, x, frame = _inputs(500, 31, 4, 300, 8.0)
+    out = _run(q, k, v, x, frame, sca.CAM_OWN_FRAME)
+    ref = torch.from_numpy(x.double().numpy() + v.double().numpy()[frame.long().numpy()]).bfloat16()
+    assert torch.equal(out, ref)
+
+
+def test_frames_outside_the_segment_keep_the_residual():
+    q, k, v, x, _ = _inputs(64, 8, 2, 301)
+    frame = torch.tensor([-3, 8, 9, 100] * 16, dtype=torch.int32)
+    for mode in (sca.CAM_OWN_FRAME, sca.CAM_UP_TO_FRAME):
+        assert torch.equal(_run(q, k, v, x, frame, mode), x)
+
+
+def test_in_place_equals_out_of_place():
+    q, k, v, x, frame = _inputs(777, 20, 16, 302)
+    a = _run(q, k, v, x, frame, sca.CAM_UP_TO_FRAME)
+    xd = x.cuda()
+    sca.camera_cross_attn(q.cuda(), k.cuda(), v.cuda(), xd, xd, frame.cuda(),
+                          sca.CAM_UP_TO_FRAME, SCALE)
+    torch.cuda.synchronize()
+    assert torch.equal(xd.cpu(), a)
+
+
+def test_repeat_is_bit_identical_and_zero_rows_launch_nothing():
+    q, k, v, x, frame = _inputs(129, 12, 2, 303)
+    a = _run(q, k, v, x, frame, sca.CAM_ALL)
+    b = _run(q, k, v, x, frame, sca.CAM_ALL)
+    assert torch.equal(a, b)
+    e = torch.empty(0, 2, D, dtype=torch.bfloat16, device="cuda")
+    sca.camera_cross_attn(e, k.cuda(), v.cuda(), e, e, None, sca.CAM_ALL, SCALE)
+    torch.cuda.synchronize()
+
+
+def test_480p_segment_sampled_rows():
+    """The bench's shape: the 12,090 video queries of a 480p segment (31
+    latent frames of 390 tokens) over its 31 camera tokens, 16 heads;
+    sampled rows against the oracle."""
+    n_q, n_cam, heads = 31 * 390, 31, 16
+    q, k, v, x, _ = _inputs(n_q, n_cam, heads, 304)
+    frame = (torch.arange(n_q, dtype=torch.int32) // 390)
+    out = _run(q, k, v, x, frame, sca.CAM_UP_TO_FRAME)
+    rows = np.unique(np.r_[0, n_q - 1, np.random.default_rng(5).choice(n_q, 256, replace=False)])
+    ref = _ref(q[rows], k, v, x[rows], frame[rows], sca.CAM_UP_TO_FRAME)
+    _check(out[rows], ref)
