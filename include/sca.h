@@ -439,7 +439,11 @@ SCA_API int sca_attn_bwd_workspace_bytes(const sca_metadata* md, int32_t heads, 
  *            NULL for SCA_CAM_ALL;
  *   k_cam, v_cam : bf16 [n_cam][heads][128] (16-byte aligned);
  *   n_q >= 0, 1 <= n_cam <= SCA_MAX_CAMERA_TOKENS, heads >= 1;
- *   softmax_scale : finite (1/sqrt(128) for the model's heads).
+ *   softmax_scale : finite (1/sqrt(128) for the model's heads);
+ *   dev_status : device int32 (or NULL); left unchanged on success, set to
+ *            SCA_ERR_DEVICE_TIMEOUT if a staged tile does not land within the
+ *            pipeline-wait limit (sca_set_pipeline_timeout_ns), the output
+ *            then incomplete.
  * S and O are accumulated in fp32, P is rounded to bf16 for its product, the
  * output is rounded once to bf16. Enqueued on `stream`; allocates nothing.
  * SCA_ERR_INVALID_ARG / SCA_ERR_MISALIGNED on bad arguments, and
@@ -450,7 +454,7 @@ enum { SCA_CAM_ALL = 0, SCA_CAM_OWN_FRAME = 1, SCA_CAM_UP_TO_FRAME = 2 };
 SCA_API int sca_camera_cross_attn(const void* q, const int32_t* q_frame, const void* k_cam,
                                   const void* v_cam, const void* x, void* out, int32_t n_q,
                                   int32_t n_cam, int32_t heads, int32_t mode,
-                                  float softmax_scale, void* stream);
+                                  float softmax_scale, int32_t* dev_status, void* stream);
 
 /* Message of the calling thread's last failure ("" if none). */
 SCA_API const char* sca_last_error(void);

@@ -727,57 +727,6 @@ int sca_kv_cache_append(sca_kv_cache* c, const sca_segment* segment, const void*
 }
 
 // ---------------------------------------------------------------------------
-// camera cross-attention
-// ---------------------------------------------------------------------------
-
-int sca_camera_cross_attn(const void* q, const int32_t* q_frame, const void* k_cam,
-                          const void* v_cam, const void* x, void* out, int32_t n_q, int32_t n_cam,
-                          int32_t heads, int32_t mode, float softmax_scale, void* stream) {
-  if (n_q < 0 || heads < 1) return fail(SCA_ERR_INVALID_ARG, "n_q must be >= 0 and heads >= 1");
-  if (n_cam < 1 || n_cam > SCA_MAX_CAMERA_TOKENS)
-    return fail(SCA_ERR_INVALID_ARG, "n_cam must be in [1, %d]", SCA_MAX_CAMERA_TOKENS);
-  if (mode != SCA_CAM_ALL && mode != SCA_CAM_OWN_FRAME && mode != SCA_CAM_UP_TO_FRAME)
-    return fail(SCA_ERR_INVALID_ARG, "unknown camera attention mode %d", mode);
-  if (!std::isfinite(softmax_scale)) return fail(SCA_ERR_INVALID_ARG, "softmax_scale must be finite");
-  if (int64_t(n_q) * heads > INT32_MAX / 128 || heads > 65535)
-    return fail(SCA_ERR_UNSUPPORTED, "too many query rows or heads");
-  if (!k_cam || !v_cam) return fail(SCA_ERR_INVALID_ARG, "null camera keys or values");
-  if (!aligned16(k_cam) || !aligned16(v_cam))
-    return fail(SCA_ERR_MISALIGNED, "camera keys and values must be 16-byte aligned");
-  if (n_q > 0) {
-    if (!q || !x || !out) return fail(SCA_ERR_INVALID_ARG, "null q, x or out");
-    if (!aligned16(q) || !aligned16(x) || !aligned16(out))
-      return fail(SCA_ERR_MISALIGNED, "q, x and out must be 16-byte aligned");
-    if (mode != SCA_CAM_ALL && !q_frame)
-      return fail(SCA_ERR_INVALID_ARG, "the frame modes need q_frame");
-    // out may be x itself; any other overlap of out with an input is refused
-    const uint64_t bytes = uint64_t(n_q) * uint64_t(heads) * SCA_HEAD_DIM * 2;
-    auto overlaps = [&](const void* p, uint64_t n) {
-      const uintptr_t a0 = reinterpret_cast<uintptr_t>(out), b0 = reinterpret_cast<uintptr_t>(p);
-      return a0 < b0 + n && b0 < a0 + bytes;
-    };
-    const uint64_t cam_bytes = uint64_t(n_cam) * uint64_t(heads) * SCA_HEAD_DIM * 2;
-    if ((out != x && overlaps(x, bytes)) || overlaps(q, bytes) || overlaps(k_cam, cam_bytes) ||
-        overlaps(v_cam, cam_bytes))
-      return fail(SCA_ERR_INVALID_ARG, "out overlaps an input (only out == x is allowed)");
-  }
-  CamArgs a{};
-  a.q = q;
-  a.q_frame = mode == SCA_CAM_ALL ? nullptr : q_frame;
-  a.k_cam = k_cam;
-  a.v_cam = v_cam;
-  a.x = x;
-  a.out = out;
-  a.n_q = n_q;
-  a.n_cam = n_cam;
-  a.heads = heads;
-  a.mode = mode;
-  a.scale_log2 = softmax_scale * 1.4426950408889634f;
-  return check_cuda(launch_camera_xattn(a, static_cast<cudaStream_t>(stream)),
-                    "camera cross-attention launch");
-}
-
-// ---------------------------------------------------------------------------
 // attention
 // ---------------------------------------------------------------------------
 
@@ -849,6 +798,65 @@ static int make_scale_map(CUtensorMap* m, const float* base, uint64_t rows, uint
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SCA_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", int(r));
   return SCA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// camera cross-attention
+// ---------------------------------------------------------------------------
+
+int sca_camera_cross_attn(const void* q, const int32_t* q_frame, const void* k_cam,
+                          const void* v_cam, const void* x, void* out, int32_t n_q, int32_t n_cam,
+                          int32_t heads, int32_t mode, float softmax_scale, int32_t* dev_status,
+                          void* stream) {
+  if (n_q < 0 || heads < 1) return fail(SCA_ERR_INVALID_ARG, "n_q must be >= 0 and heads >= 1");
+  if (n_cam < 1 || n_cam > SCA_MAX_CAMERA_TOKENS)
+    return fail(SCA_ERR_INVALID_ARG, "n_cam must be in [1, %d]", SCA_MAX_CAMERA_TOKENS);
+  if (mode != SCA_CAM_ALL && mode != SCA_CAM_OWN_FRAME && mode != SCA_CAM_UP_TO_FRAME)
+    return fail(SCA_ERR_INVALID_ARG, "unknown camera attention mode %d", mode);
+  if (!std::isfinite(softmax_scale)) return fail(SCA_ERR_INVALID_ARG, "softmax_scale must be finite");
+  if (int64_t(n_q) * heads > INT32_MAX / 128 || heads > 65535)
+    return fail(SCA_ERR_UNSUPPORTED, "too many query rows or heads");
+  if (!k_cam || !v_cam) return fail(SCA_ERR_INVALID_ARG, "null camera keys or values");
+  if (!aligned16(k_cam) || !aligned16(v_cam))
+    return fail(SCA_ERR_MISALIGNED, "camera keys and values must be 16-byte aligned");
+  if (n_q > 0) {
+    if (!q || !x || !out) return fail(SCA_ERR_INVALID_ARG, "null q, x or out");
+    if (!aligned16(q) || !aligned16(x) || !aligned16(out))
+      return fail(SCA_ERR_MISALIGNED, "q, x and out must be 16-byte aligned");
+    if (mode != SCA_CAM_ALL && !q_frame)
+      return fail(SCA_ERR_INVALID_ARG, "the frame modes need q_frame");
+    // out may be x itself; any other overlap of out with an input is refused
+    const uint64_t bytes = uint64_t(n_q) * uint64_t(heads) * SCA_HEAD_DIM * 2;
+    auto overlaps = [&](const void* p, uint64_t n) {
+      const uintptr_t a0 = reinterpret_cast<uintptr_t>(out), b0 = reinterpret_cast<uintptr_t>(p);
+      return a0 < b0 + n && b0 < a0 + bytes;
+    };
+    const uint64_t cam_bytes = uint64_t(n_cam) * uint64_t(heads) * SCA_HEAD_DIM * 2;
+    if ((out != x && overlaps(x, bytes)) || overlaps(q, bytes) || overlaps(k_cam, cam_bytes) ||
+        overlaps(v_cam, cam_bytes))
+      return fail(SCA_ERR_INVALID_ARG, "out overlaps an input (only out == x is allowed)");
+  }
+  CamArgs a{};
+  a.q_frame = mode == SCA_CAM_ALL ? nullptr : q_frame;
+  a.n_q = n_q;
+  a.n_cam = n_cam;
+  a.heads = heads;
+  a.mode = mode;
+  a.scale_log2 = softmax_scale * 1.4426950408889634f;
+  a.status = dev_status;
+  a.timeout_ns = g_pipeline_timeout_ns;
+  if (n_q == 0) return SCA_OK;
+  CamMaps maps;
+  const uint64_t row = uint64_t(heads) * SCA_HEAD_DIM * 2;
+  const uint32_t box = uint32_t(camera_box_rows(n_cam));
+  int rc = make_map(&maps.q, q, uint64_t(heads), uint64_t(n_q), SCA_HEAD_DIM * 2, row, 1, 128);
+  if (!rc) rc = make_map(&maps.x, x, uint64_t(heads), uint64_t(n_q), SCA_HEAD_DIM * 2, row, 1, 128);
+  if (!rc) rc = make_map(&maps.out, out, uint64_t(heads), uint64_t(n_q), SCA_HEAD_DIM * 2, row, 1, 128);
+  if (!rc) rc = make_map(&maps.k, k_cam, uint64_t(heads), uint64_t(n_cam), SCA_HEAD_DIM * 2, row, 1, box);
+  if (!rc) rc = make_map(&maps.v, v_cam, uint64_t(heads), uint64_t(n_cam), SCA_HEAD_DIM * 2, row, 1, box);
+  if (rc) return rc;
+  return check_cuda(launch_camera_xattn(maps, a, static_cast<cudaStream_t>(stream)),
+                    "camera cross-attention launch");
 }
 
 // ---------------------------------------------------------------------------

@@ -102,7 +102,8 @@ _SIGS = {
     "sca_action_causal_attn_bwd": [_P, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_float,
                                    _P, ctypes.c_uint64, _P, _P],
     "sca_attn_bwd_workspace_bytes": [_P, _i32, ctypes.POINTER(ctypes.c_uint64)],
-    "sca_camera_cross_attn": [_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, ctypes.c_float, _P],
+    "sca_camera_cross_attn": [_P, _P, _P, _P, _P, _P, _i32, _i32, _i32, _i32, ctypes.c_float, _P,
+                              _P],
     "sca_attn_plan": [_P, _i32, _pi32, _pi32, _pi32],
     "sca_attn_plan_for_sms": [_P, _i32, _i32, _pi32, _pi32, _pi32, ctypes.POINTER(ctypes.c_uint64)],
     "sca_set_split_override": [_i32],
@@ -406,11 +407,12 @@ def action_causal_attn_bwd(md: Metadata, heads: int, q, k, v, o, lse, d_o, dq, d
 
 
 def camera_cross_attn(q, k_cam, v_cam, x, out, q_frame=None, mode: int = CAM_ALL,
-                      softmax_scale: float = 128 ** -0.5, stream=None) -> None:
+                      softmax_scale: float = 128 ** -0.5, dev_status=None, stream=None) -> None:
     """out = x + the camera cross-attention of queries ``q`` over one
     segment's camera tokens (see include/sca.h). ``q``, ``x``, ``out``: bf16
     [n_q, heads, 128] (``out`` may be ``x``); ``k_cam``, ``v_cam``: bf16
-    [n_cam, heads, 128]; ``q_frame``: int32 [n_q] or None (SCA_CAM_ALL)."""
+    [n_cam, heads, 128]; ``q_frame``: int32 [n_q] or None (SCA_CAM_ALL);
+    ``dev_status``: device int32 or None."""
     n_q, heads = int(q.shape[0]), int(q.shape[1])
     if tuple(x.shape) != tuple(q.shape) or tuple(out.shape) != tuple(q.shape):
         raise ValueError("q, x and out must have the same shape [n_q, heads, 128]")
@@ -418,7 +420,7 @@ def camera_cross_attn(q, k_cam, v_cam, x, out, q_frame=None, mode: int = CAM_ALL
         raise ValueError("k_cam and v_cam must be [n_cam, heads, 128]")
     _check(_lib.sca_camera_cross_attn(_ptr(q), _ptr(q_frame), _ptr(k_cam), _ptr(v_cam), _ptr(x),
                                       _ptr(out), n_q, int(k_cam.shape[0]), heads, int(mode),
-                                      float(softmax_scale), _stream(stream)))
+                                      float(softmax_scale), _ptr(dev_status), _stream(stream)))
 
 
 def attn_int8_scratch_bytes(md: Metadata, heads: int) -> int:

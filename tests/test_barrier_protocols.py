@@ -12,7 +12,8 @@ or a wait that sees its barrier two phases away.
 
 Pipelines: the attention forward's K/V ring with the INT8 cache's staged code
 slots (a prefix of cache tiles dequantised into the ring, then current tiles
-loaded directly), and the backward's dQ and dK/dV kernels.
+loaded directly), the backward's dQ and dK/dV kernels, and the camera
+cross-attention's per-warp ring of staged row tiles.
 """
 import random
 
@@ -462,3 +463,154 @@ def test_dkdv_region_hazards_would_be_caught(mutation):
         for n in range(2, 8):
             for seed in range(40):
                 scope["backward_dkdv"](n, seed)
+
+
+# ---------------------------------------------------------------------------
+# camera cross-attention: a producer streams each 128-row tile's q (ring of
+# qs stages) and, once per run of tiles of one head, that head's camera K/V
+# (2 entries); one MMA thread issues S_k into tensor-memory buffer k % 2,
+# then P V of the previous tile; the epilogue warpgroup k % 2 takes tile k
+# (softmax, then x + O / l over x); a store thread sends each finished tile
+# back and then loads the x of tile k + xs into the freed stage (it also arms
+# the first xs)
+# ---------------------------------------------------------------------------
+
+def camera_pipeline(heads, qs, xs, seed, mutation=None):
+    n = len(heads)
+    bars = {("kvfull", e): Bar(1) for e in range(2)}
+    bars.update({("kvempty", e): Bar(1) for e in range(2)})
+    bars.update({("qfull", s): Bar(1) for s in range(qs)})
+    bars.update({("qempty", s): Bar(1) for s in range(qs)})
+    bars.update({("xfull", s): Bar(1) for s in range(xs)})
+    for j in range(2):
+        for name in ("S", "P", "O", "Store"):
+            bars[(name, j)] = Bar(1)
+    kv_owner, q_owner, x_owner = {}, {}, {}
+    s_tile, o_tile = {}, {}
+    pv_issued, o_read = set(), set()
+
+    def producer():
+        run, hprev = -1, None
+        for k, h in enumerate(heads):
+            if h != hprev:
+                if run >= 1 and mutation != "no kv wait":
+                    u = (run + 1) // 2 - 1
+                    yield wait(("kvempty", (run + 1) & 1), u & 1, u)
+                run, hprev = run + 1, h
+                e = run & 1
+                assert kv_owner.get(e) is None, "K/V entry refilled while in use"
+                kv_owner[e] = run
+                bars[("kvfull", e)].expect(4)
+                for _ in range(4):
+                    yield ("copy", ("kvfull", e), 1)
+            sq = k % qs
+            if k >= qs:
+                yield wait(("qempty", sq), (k // qs - 1) & 1, k // qs - 1)
+            assert q_owner.get(sq) is None, "q stage refilled while in use"
+            q_owner[sq] = k
+            bars[("qfull", sq)].expect(2)
+            yield ("copy", ("qfull", sq), 1)
+            yield ("copy", ("qfull", sq), 1)
+
+    def mma():
+        def pv(i, ri, last):
+            j = i & 1
+            yield wait(("P", j), (i >> 1) & 1, i >> 1)
+            assert s_tile.get(j) == i and kv_owner.get(ri & 1) == ri
+            assert i < 2 or (i - 2) in o_read, "O buffer overwritten before it was read"
+            o_tile[j] = i
+            pv_issued.add(i)
+            bars[("O", j)].arrive()
+            if last:
+                kv_owner[ri & 1] = None
+                bars[("kvempty", ri & 1)].arrive()
+
+        run, hprev, run_prev = -1, None, 0
+        for k, h in enumerate(heads):
+            if h != hprev:
+                run, hprev = run + 1, h
+                yield wait(("kvfull", run & 1), (run >> 1) & 1, run >> 1)
+            sq, j = k % qs, k & 1
+            yield wait(("qfull", sq), (k // qs) & 1, k // qs)
+            assert q_owner.get(sq) == k and kv_owner.get(run & 1) == run
+            assert k < 2 or (k - 2) in pv_issued, "S buffer overwritten before its P was used"
+            s_tile[j] = k
+            q_owner[sq] = None
+            bars[("qempty", sq)].arrive()
+            bars[("S", j)].arrive()
+            if k >= 1:
+                yield from pv(k - 1, run_prev, h != heads[k - 1])
+            run_prev = run
+        if n:
+            yield from pv(n - 1, run_prev, True)
+
+    def epilogue(wg):
+        for k in range(wg, n, 2):
+            m, sx = k >> 1, k % xs
+            yield wait(("S", wg), m & 1, m)
+            assert s_tile.get(wg) == k
+            yield ("work",)
+            bars[("P", wg)].arrive()
+            yield wait(("O", wg), m & 1, m)
+            yield wait(("xfull", sx), (k // xs) & 1, k // xs)
+            assert o_tile.get(wg) == k and x_owner.get(sx) == k, "epilogue reads another tile"
+            yield ("work",)
+            o_read.add(k)
+            bars[("Store", wg)].arrive()
+
+    def store():
+        def load_x(k):
+            sx = k % xs
+            assert x_owner.get(sx) is None, "x stage refilled while in use"
+            x_owner[sx] = k
+            bars[("xfull", sx)].expect(2)
+            return [("copy", ("xfull", sx), 1), ("copy", ("xfull", sx), 1)]
+
+        loaded = 0
+        while loaded < min(n, xs):
+            yield from load_x(loaded)
+            loaded += 1
+        for k in range(n):
+            sx = k % xs
+            if mutation == "x before store" and loaded < n:
+                x_owner[sx] = None
+                yield from load_x(loaded)
+                loaded += 1
+            yield wait(("Store", k & 1), (k >> 1) & 1, k >> 1)
+            assert k in o_read
+            if mutation != "x before store":
+                assert x_owner.get(sx) == k
+                yield ("work",)
+                x_owner[sx] = None
+                if loaded < n:
+                    yield from load_x(loaded)
+                    loaded += 1
+
+    run({"producer": producer(), "mma": mma(), "epi0": epilogue(0), "epi1": epilogue(1),
+         "store": store()}, bars, seed)
+
+
+def _camera_heads(rng):
+    """Head of every tile of one CTA's range: runs of 1 to 12 tiles."""
+    heads, h = [], rng.randint(0, 3)
+    for _ in range(rng.randint(1, 4)):
+        heads += [h] * rng.randint(1, 12)
+        h += 1
+    return heads
+
+
+@pytest.mark.parametrize("qs, xs", [(2, 3), (2, 4), (3, 3)])
+def test_camera_pipeline(qs, xs):
+    """The shipped depths (2 q stages, 3 or 4 x stages) and another; ranges
+    of one tile, of one head, and of several heads."""
+    for seed in range(60):
+        camera_pipeline(_camera_heads(random.Random(seed)), qs, xs, seed)
+
+
+@pytest.mark.parametrize("mutation", ["x before store", "no kv wait"])
+def test_camera_missing_waits_would_be_caught(mutation):
+    """(O needs no free barrier: a warpgroup arrives at P of tile i only after
+    it has read O of tile i - 2, which the model checks on every P V.)"""
+    with pytest.raises(AssertionError):
+        for seed in range(60):
+            camera_pipeline(_camera_heads(random.Random(seed)), 2, 3, seed, mutation)

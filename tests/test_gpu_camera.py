@@ -39,8 +39,10 @@ def _inputs(n_q, n_cam, heads, seed, sharp=1.0):
 def _run(q, k, v, x, frame, mode, out=None):
     qd, kd, vd, xd, fd = (t.cuda() for t in (q, k, v, x, frame))
     od = torch.empty_like(xd) if out is None else out
-    sca.camera_cross_attn(qd, kd, vd, xd, od, fd, mode, SCALE)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sca.camera_cross_attn(qd, kd, vd, xd, od, fd, mode, SCALE, st)
     torch.cuda.synchronize()
+    assert int(st.item()) == 0
     return od.cpu()
 
 
@@ -116,3 +118,55 @@ def test_480p_segment_sampled_rows():
     rows = np.unique(np.r_[0, n_q - 1, np.random.default_rng(5).choice(n_q, 256, replace=False)])
     ref = _ref(q[rows], k, v, x[rows], frame[rows], sca.CAM_UP_TO_FRAME)
     _check(out[rows], ref)
+
+
+@pytest.mark.parametrize("n_cam, mode", [(9, 1), (40, 2), (64, 0), (64, 2)])
+def test_long_ranges_of_tiles_per_cta(n_cam, mode):
+    """Enough rows that every CTA streams several 128-row tiles, across head
+    changes, for each width of the camera tile; sampled rows."""
+    n_q, heads = 9000, 16
+    q, k, v, x, _ = _inputs(n_q, n_cam, heads, 400 + n_cam + mode)
+    frame = (torch.arange(n_q, dtype=torch.int32) * n_cam // n_q)
+    out = _run(q, k, v, x, frame, mode)
+    rows = np.unique(np.r_[0, 127, 128, n_q - 1,
+                           np.random.default_rng(n_cam).choice(n_q, 200, replace=False)])
+    _check(out[rows], _ref(q[rows], k, v, x[rows], frame[rows], mode))
+
+
+def test_unaligned_frame_index():
+    """A q_frame view one element into its buffer (not 16-byte aligned)."""
+    q, k, v, x, frame = _inputs(333, 24, 4, 305)
+    buf = torch.zeros(frame.numel() + 1, dtype=torch.int32)
+    buf[1:] = frame
+    fd = buf.cuda()[1:]
+    assert fd.data_ptr() % 16 != 0
+    od = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    sca.camera_cross_attn(q.cuda(), k.cuda(), v.cuda(), x.cuda(), od, fd, sca.CAM_UP_TO_FRAME,
+                          SCALE)
+    torch.cuda.synchronize()
+    _check(od.cpu(), _ref(q, k, v, x, frame, sca.CAM_UP_TO_FRAME))
+
+
+
+def test_calls_replay_from_a_cuda_graph():
+    """Captured in a CUDA graph (each call with its own tensor maps), the
+    calls replay to the eager results bit for bit."""
+    q, k, v, x, frame = _inputs(1000, 31, 16, 307)
+    x2 = x.flip(0).contiguous()
+    eager = [_run(q, k, v, xx, frame, sca.CAM_UP_TO_FRAME) for xx in (x, x2)]
+    qd, kd, vd, fd = q.cuda(), k.cuda(), v.cuda(), frame.cuda()
+    xs = [x.cuda(), x2.cuda()]
+    outs = [torch.empty_like(xs[0]) for _ in range(2)]
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+        for xx, oo in zip(xs, outs):
+            sca.camera_cross_attn(qd, kd, vd, xx, oo, fd, sca.CAM_UP_TO_FRAME, SCALE, st,
+                                  torch.cuda.current_stream().cuda_stream)
+    for o in outs:
+        o.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for o, e in zip(outs, eager):
+        assert torch.equal(o.cpu(), e)
