@@ -656,12 +656,16 @@ __global__ void __launch_bounds__(threads_for(kInt8), 1)
 #pragma unroll
           for (int i = 0; i < 128; ++i) x[i] = ((vis[i >> 5] >> (i & 31)) & 1u) ? x[i] : -INFINITY;
         }
+        // row max in four chains: x[0..3], then x[4..123] two at a time,
+        // then x[124..127]
         float m4[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-        for (int i = 4; i < 128; i += 8) {
+        for (int i = 4; i < 124; i += 8) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) m4[k] = max3(m4[k], x[i + k], x[i + 4 + k]);
         }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) m4[k] = fmaxf(m4[k], x[124 + k]);
         const float mx = max3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
         // The running max only moves when it grows by more than the threshold
         // (exact: l and O share the stale max until the final division).
