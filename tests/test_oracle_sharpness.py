@@ -6,7 +6,9 @@ through ``monkeypatch``, undone after the case): a dropped term, a wrong
 sign, an off-by-one window end, a transposed or swapped operand, a wrong
 rounding. It then runs the pins of that part of the oracle and requires at
 least one of them to fail an assertion. The unmodified oracle passes every
-pin (the rest of the suite).
+pin (the rest of the suite); for the camera cross-attention, whose mistakes
+are planted in a restatement of the oracle, the restatement left correct is
+shown to pass the same pins.
 """
 import functools
 import os
@@ -17,11 +19,13 @@ import pytest
 from oracle import attention as oattn
 from oracle import backward as obwd
 from oracle import cache as ocache
+from oracle import camera as ocam
 from oracle import rule as orule
 from oracle import schedule as osched
 from segment_causal_masked_b200 import workloads as W
 from tests import test_oracle_attention as ta
 from tests import test_oracle_backward as tb
+from tests import test_oracle_camera as tc
 from tests import test_oracle_int8 as ti
 from tests import test_oracle_rule as tr
 
@@ -385,3 +389,116 @@ def _one_tiling(layout):
 def test_schedule_mistake_is_caught(attr, fn, monkeypatch):
     monkeypatch.setattr(osched, attr, fn)
     assert _first_failure(_schedule_pins()) is not None
+
+
+# ---------------------------------------------------------------------------
+# planted mistakes: camera cross-attention
+# ---------------------------------------------------------------------------
+
+def _camera_pins():
+    pins = [_p(tc.test_matches_torch_sdpa, mode, n_cam, sharp)
+            for mode in (ocam.CAM_ALL, ocam.CAM_UP_TO_FRAME) for n_cam in (1, 7, 31)
+            for sharp in (1.0, 6.0)]
+    return pins + [tc.test_own_frame_adds_that_frames_value_row, tc.test_single_camera_token,
+                   tc.test_equal_keys_give_the_mean_of_the_visible_values,
+                   tc.test_frames_outside_the_segment_keep_the_residual,
+                   tc.test_all_mode_ignores_the_order_of_camera_tokens, tc.test_visibility_sets]
+
+
+_vis = ocam.visible_camera_tokens
+_cxa = ocam.camera_cross_attention
+
+
+def _vis_with(fn):
+    def vis(q_frame, n_cam, mode):
+        q_frame = np.asarray(q_frame, dtype=np.int64)
+        if mode == ocam.CAM_ALL:
+            return _vis(q_frame, n_cam, mode)
+        if mode not in (ocam.CAM_OWN_FRAME, ocam.CAM_UP_TO_FRAME):
+            raise ValueError("unknown camera attention mode")
+        return fn(q_frame[:, None], np.arange(n_cam)[None, :], n_cam, mode)
+    return vis
+
+
+CAMERA_VISIBILITY_MISTAKES = {
+    "own frame off by one": _vis_with(
+        lambda qf, f, n, mode: ((qf >= 0) & (qf < n)) & ((f == qf + 1) if mode == ocam.CAM_OWN_FRAME
+                                                         else (f <= qf))),
+    "frames up to the own one, exclusive": _vis_with(
+        lambda qf, f, n, mode: ((qf >= 0) & (qf < n)) & ((f == qf) if mode == ocam.CAM_OWN_FRAME
+                                                         else (f < qf))),
+    "frames outside the segment see tokens": _vis_with(
+        lambda qf, f, n, mode: (f == qf) if mode == ocam.CAM_OWN_FRAME else (f <= qf)),
+    "every token for the whole segment": lambda q_frame, n_cam, mode: np.ones(
+        (np.asarray(q_frame).shape[0], n_cam), dtype=bool),
+}
+
+
+def test_camera_visibility_restatement_without_a_mistake_passes(monkeypatch):
+    monkeypatch.setattr(ocam, "visible_camera_tokens", _vis_with(
+        lambda qf, f, n, mode: ((qf >= 0) & (qf < n)) & ((f == qf) if mode == ocam.CAM_OWN_FRAME
+                                                         else (f <= qf))))
+    assert _first_failure(_camera_pins()) is None
+
+
+@pytest.mark.parametrize("name", list(CAMERA_VISIBILITY_MISTAKES))
+def test_camera_visibility_mistake_is_caught(name, monkeypatch):
+    monkeypatch.setattr(ocam, "visible_camera_tokens", CAMERA_VISIBILITY_MISTAKES[name])
+    assert _first_failure(_camera_pins()) is not None, name
+
+
+def _camera_with(mistake):
+    def f(q, k_cam, v_cam, x, q_frame, mode, scale):
+        q = np.asarray(q, dtype=np.float64)
+        k = np.asarray(k_cam, dtype=np.float64)
+        v = np.asarray(v_cam, dtype=np.float64)
+        x = np.asarray(x, dtype=np.float64)
+        vis = ocam.visible_camera_tokens(q_frame, k.shape[0], mode)
+        return mistake(q, k, v, x, vis, scale)
+    return f
+
+
+def _camera_attn(q, k, v, x, vis, scale, masked_value=-np.inf, residual=True, axis=1):
+    out = np.array(x) if residual else np.zeros_like(x)
+    for h in range(q.shape[1]):
+        s = (q[:, h, :] @ k[:, h, :].T) * scale
+        s = np.where(vis, s, masked_value)
+        m = s.max(axis=axis, keepdims=True, initial=-np.inf)
+        m = np.where(np.isfinite(m), m, 0.0)
+        e = np.exp(s - m)
+        z = e.sum(axis=axis, keepdims=True)
+        p = np.divide(e, z, out=np.zeros_like(e), where=z > 0)
+        out[:, h, :] += p @ v[:, h, :]
+    return out
+
+
+CAMERA_MISTAKES = {
+    "residual not added": _camera_with(lambda q, k, v, x, vis, scale: _camera_attn(
+        q, k, v, x, vis, scale, residual=False)),
+    "scale dropped": _camera_with(lambda q, k, v, x, vis, scale: _camera_attn(q, k, v, x, vis, 1.0)),
+    "keys used as values": _camera_with(lambda q, k, v, x, vis, scale: _camera_attn(
+        q, k, k, x, vis, scale)),
+    "hidden tokens scored 0 instead of -inf": _camera_with(
+        lambda q, k, v, x, vis, scale: _camera_attn(q, k, v, x, vis, scale, masked_value=0.0)),
+    "softmax over the queries": _camera_with(lambda q, k, v, x, vis, scale: _camera_attn(
+        q, k, v, x, vis, scale, axis=0)),
+    "queries that see nothing get the mean value": _camera_with(
+        lambda q, k, v, x, vis, scale: np.where(
+            vis.any(axis=1)[:, None, None], _camera_attn(q, k, v, x, vis, scale),
+            x + v.mean(axis=0)[None])),
+}
+
+
+def test_camera_restatement_without_a_mistake_passes(monkeypatch):
+    """Control: the restatement the mistakes are planted in, left correct,
+    passes every camera pin (so a caught mistake is the mistake's doing)."""
+    monkeypatch.setattr(ocam, "camera_cross_attention",
+                        _camera_with(lambda q, k, v, x, vis, scale: _camera_attn(q, k, v, x, vis,
+                                                                                  scale)))
+    assert _first_failure(_camera_pins()) is None
+
+
+@pytest.mark.parametrize("name", list(CAMERA_MISTAKES))
+def test_camera_mistake_is_caught(name, monkeypatch):
+    monkeypatch.setattr(ocam, "camera_cross_attention", CAMERA_MISTAKES[name])
+    assert _first_failure(_camera_pins()) is not None, name
