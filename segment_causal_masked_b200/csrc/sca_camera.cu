@@ -30,6 +30,10 @@
 // * A store thread writes each finished tile back with a TMA tensor store and,
 //   once the store has read the stage, loads the x of the tile that uses the
 //   stage next.
+// * Launched as a programmatic dependent of the work before it on the stream:
+//   the CTAs allocate tensor memory and set up their barriers while that work
+//   finishes, then wait for it (griddepcontrol.wait) before any global memory
+//   access; each call lets the next one launch early in the same way.
 // * Every wait is bounded: a wait that runs out sets SCA_ERR_DEVICE_TIMEOUT in
 //   the status word, every role lets its own copies and products in flight
 //   complete, and the CTA frees its tensor memory and exits.
@@ -190,6 +194,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the next launch on the stream may be scheduled now; this one reads and
+  // writes global memory only once the work before it has completed
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
@@ -463,8 +471,17 @@ cudaError_t launch_nf(const CamMaps& m, const CamArgs& a, cudaStream_t stream, i
   }
   const int64_t total = int64_t((a.n_q + 127) / 128) * a.heads;
   const int grid = int(total < sms ? total : sms);
-  camera_xattn_kernel<NF><<<grid, kThreads, smem, stream>>>(m.q, m.x, m.out, m.k, m.v, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, camera_xattn_kernel<NF>, m.q, m.x, m.out, m.k, m.v, a);
 }
 
 // SM count of each device, read once (0: not read yet)
