@@ -445,7 +445,10 @@ SCA_API int sca_attn_bwd_workspace_bytes(const sca_metadata* md, int32_t heads, 
  *            pipeline-wait limit (sca_set_pipeline_timeout_ns), the output
  *            then incomplete.
  * S and O are accumulated in fp32, P is rounded to bf16 for its product, the
- * output is rounded once to bf16. Enqueued on `stream`; allocates nothing.
+ * output is rounded once to bf16. Enqueued on `stream` as a programmatic
+ * dependent launch: the kernel may start its set-up while earlier work on the
+ * stream finishes, but reads and writes memory only after that work is
+ * complete, so the ordering is that of a plain launch. Allocates nothing.
  * SCA_ERR_INVALID_ARG / SCA_ERR_MISALIGNED on bad arguments, and
  * SCA_ERR_UNSUPPORTED past 65,535 heads or 2^31 elements of q (nothing is
  * launched then). */

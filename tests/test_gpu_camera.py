@@ -65,7 +65,7 @@ def test_matches_oracle(mode, n_cam):
     _check(_run(q, k, v, x, frame, mode), _ref(q, k, v, x, frame, mode))
 
 
-@pytest.mark.parametrize("n_q", [1, 15, 16, 17, 2048])
+@pytest.mark.parametrize("n_q", [1, 15, 16, 17, 127, 128, 129, 255, 256, 257, 2048])
 @pytest.mark.parametrize("sharp", [1.0, 8.0])
 def test_ragged_rows_and_sharp_scores(n_q, sharp):
     q, k, v, x, frame = _inputs(n_q, 31, 16, 200 + n_q, sharp)
