@@ -29,7 +29,11 @@
 //   tile, with packed two-lane fp32 arithmetic.
 // * A store thread writes each finished tile back with a TMA tensor store and,
 //   once the store has read the stage, loads the x of the tile that uses the
-//   stage next.
+//   stage next. Each warpgroup has x stages of its own (and two store
+//   barriers), so that every barrier's phases are waited for in order by the
+//   one warpgroup that uses it: with one ring shared by both, a warpgroup
+//   could wait on a stage's next phase before the other one's had completed,
+//   and a parity wait would take the incomplete phase for the awaited one.
 // * Launched as a programmatic dependent of the work before it on the stream:
 //   the CTAs allocate tensor memory and set up their barriers while that work
 //   finishes, then wait for it (griddepcontrol.wait) before any global memory
@@ -58,10 +62,10 @@ constexpr int kHalf = 128 * 128;        // one 64-column half of a 128-row tile
 constexpr int kTile = 2 * kHalf;        // a 128-row tile of q or x
 template <int NF>  // camera tokens rounded up to 16
 struct CamLayout {
-  // q runs two tiles ahead of the products where shared memory allows: the
-  // MMA thread issues S of tile k + 1 before P V of tile k
-  static constexpr int kQStages = NF <= 32 ? 3 : 2;
-  static constexpr int kXStages = 3;
+  // x stages per epilogue warpgroup (2 where shared memory allows), q stages
+  static constexpr int kXPerWg = NF <= 32 ? 2 : 1;
+  static constexpr int kXStages = 2 * kXPerWg;
+  static constexpr int kQStages = NF <= 32 ? 2 : 3;
   static constexpr int kKVHalf = NF * 128;           // a 64-column half of K or V
   static constexpr int kKV = 4 * kKVHalf;            // K and V of one head
   // barriers (8 bytes each) and control words in the first 1024 bytes
@@ -69,7 +73,7 @@ struct CamLayout {
                        kBarQEmpty = kBarQFull + kQStages, kBarXFull = kBarQEmpty + kQStages,
                        kBarS = kBarXFull + kXStages,
                        kBarP = kBarS + 2, kBarO = kBarP + 2, kBarStore = kBarO + 2,
-                       kBarDrain = kBarStore + 2,
+                       kBarDrain = kBarStore + 4,
                        kNumBars = kBarDrain + 1;
   static constexpr int kOffCtl = 1000, kOffTmem = 1008;
   static constexpr int kOffQ = 1024;
@@ -157,7 +161,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const CamArgs a) {
   using L = CamLayout<NF>;
-  constexpr int kXS = L::kXStages, kQStages = L::kQStages;
+  constexpr int kXS = L::kXStages, kQStages = L::kQStages, kXPerWg = L::kXPerWg;
+  // tile k, the m-th tile (m = k / 2) of warpgroup k % 2: its x stage, the
+  // use of that stage it is, and its store barrier
+  auto x_stage = [&](int k) { return (k & 1) * kXPerWg + (k >> 1) % kXPerWg; };
+  auto x_use = [&](int k) { return (k >> 1) / kXPerWg; };
+  auto store_bar = [&](int k) { return L::kBarStore + 2 * (k & 1) + ((k >> 1) & 1); };
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -302,20 +311,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ store
     if (lane == 0) {
       auto load_x = [&](int k) {
-        const int sx = k % kXS;
+        const int sx = x_stage(k);
         const uint32_t dx = sbase + L::kOffX + uint32_t(sx) * kTile;
         mbar_expect_tx(bar(L::kBarXFull + sx), uint32_t(kTile));
         tma_load_3d(dx, &tm_x, bar(L::kBarXFull + sx), 0, head_of(k), row0_of(k));
         tma_load_3d(dx + kHalf, &tm_x, bar(L::kBarXFull + sx), 64, head_of(k), row0_of(k));
       };
+      // the next tile in tile k's stage is k + kXS (kXPerWg tiles of the same
+      // warpgroup later); x loads go out in tile order
       int loaded = 0;  // x of tiles 0 .. loaded-1 armed
       for (; loaded < n && loaded < kXS; ++loaded) load_x(loaded);
       bool stored = false;
       for (int k = 0; k < n; ++k) {
-        const int j = k & 1, sx = k % kXS;
-        if (!wait_bar(bar(L::kBarStore + j), uint32_t(k >> 1) & 1u, ctl, a.status, a.timeout_ns))
+        if (!wait_bar(bar(store_bar(k)), uint32_t(k >> 2) & 1u, ctl, a.status, a.timeout_ns))
           break;
-        const uint32_t src = sbase + L::kOffX + uint32_t(sx) * kTile;
+        const uint32_t src = sbase + L::kOffX + uint32_t(x_stage(k)) * kTile;
         tma_store_3d(&tm_out, src, 0, head_of(k), row0_of(k));
         tma_store_3d(&tm_out, src + kHalf, 64, head_of(k), row0_of(k));
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
@@ -325,10 +335,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (loaded < n) load_x(loaded++);
       }
       // the output writes are complete, and every x copy armed has landed,
-      // before the CTA exits
+      // before the CTA exits (the last kXS tiles armed are in distinct stages)
       if (stored) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
       for (int i = loaded - kXS < 0 ? 0 : loaded - kXS; i < loaded; ++i)
-        wait_drain(bar(L::kBarXFull + i % kXS), uint32_t(i / kXS) & 1u);
+        wait_drain(bar(L::kBarXFull + x_stage(i)), uint32_t(x_use(i)) & 1u);
     }
     __syncwarp();
   } else {
@@ -400,8 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // x of the row from the staged tile (it has usually landed long before
       // O): dims 8 q .. 8 q + 7 are the 16-byte chunk q & 7 of half q >> 3,
       // swizzled by r & 7
-      const int sx = k % kXS;
-      ok = wait_bar(bar(L::kBarXFull + sx), uint32_t(k / kXS) & 1u, ctl, a.status, a.timeout_ns);
+      const int sx = x_stage(k);
+      ok = wait_bar(bar(L::kBarXFull + sx), uint32_t(x_use(k)) & 1u, ctl, a.status, a.timeout_ns);
       if (!__all_sync(0xFFFFFFFFu, ok)) {
         ok = false;
         break;
@@ -445,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // the row is written: the store thread sends the tile once all 128 are
       fence_proxy_async_smem();
-      mbar_arrive(bar(L::kBarStore + wg));
+      mbar_arrive(bar(store_bar(k)));
     }
   }
 

@@ -170,3 +170,31 @@ def test_calls_replay_from_a_cuda_graph():
     assert int(st.item()) == 0
     for o, e in zip(outs, eager):
         assert torch.equal(o.cpu(), e)
+
+
+def test_pipeline_timeout_aborts_cleanly():
+    """With the pipeline-wait limit at 0 a role gives up at its first wait
+    that is not already complete: the status word reads
+    SCA_ERR_DEVICE_TIMEOUT, every role lets its own copies and products land
+    before the CTA frees its tensor memory and exits, and the device keeps
+    answering: with the default limit back the next call is right. (A
+    try-wait may itself block until the phase completes, so the call is
+    repeated until one of them gives up.)"""
+    q, k, v, x, frame = _inputs(32768, 31, 16, 306)
+    qd, kd, vd, xd, fd = (t.cuda() for t in (q, k, v, x, frame))
+    od = torch.empty_like(xd)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    try:
+        sca.set_pipeline_timeout_ns(0)
+        for _ in range(10):
+            sca.camera_cross_attn(qd, kd, vd, xd, od, fd, sca.CAM_UP_TO_FRAME, SCALE, st)
+            torch.cuda.synchronize()
+            if int(st.item()) != 0:
+                break
+    finally:
+        sca.set_pipeline_timeout_ns(2_000_000_000)
+    assert int(st.item()) == sca.ERR_DEVICE_TIMEOUT
+    assert float((torch.ones(4, device="cuda") * 2).sum().item()) == 8.0
+    rows = np.arange(0, 32768, 61)
+    out = _run(q, k, v, x, frame, sca.CAM_UP_TO_FRAME)
+    _check(out[rows], _ref(q[rows], k, v, x[rows], frame[rows], sca.CAM_UP_TO_FRAME))
