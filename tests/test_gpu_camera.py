@@ -198,3 +198,21 @@ def test_pipeline_timeout_aborts_cleanly():
     rows = np.arange(0, 32768, 61)
     out = _run(q, k, v, x, frame, sca.CAM_UP_TO_FRAME)
     _check(out[rows], _ref(q[rows], k, v, x[rows], frame[rows], sca.CAM_UP_TO_FRAME))
+
+
+@pytest.mark.parametrize("mode", [sca.CAM_OWN_FRAME, sca.CAM_UP_TO_FRAME])
+def test_random_frames_over_many_tiles_per_cta(mode):
+    """Random frames (a stale row rarely matches) with 28 tiles of 128 rows
+    per CTA, three calls: a warp that read another tile's x (the race of a
+    shared x-stage ring) makes whole 32-row blocks wrong in some calls."""
+    q, k, v, x, frame = _inputs(32768, 31, 16, 308 + mode)
+    rows = np.arange(0, 32768, 37)
+    ref = _ref(q[rows], k, v, x[rows], frame[rows], mode)
+    qd, kd, vd, xd, fd = (t.cuda() for t in (q, k, v, x, frame))
+    for _ in range(3):
+        od = torch.empty_like(xd)
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        sca.camera_cross_attn(qd, kd, vd, xd, od, fd, mode, SCALE, st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        _check(od.cpu()[rows], ref)
