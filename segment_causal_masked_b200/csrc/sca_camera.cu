@@ -29,7 +29,7 @@
 //   tile, with packed two-lane fp32 arithmetic.
 // * A store thread writes each finished tile back with a TMA tensor store and,
 //   once the store has read the stage, loads the x of the tile that uses the
-//   stage next. Each warpgroup has x stages of its own (and two store
+//   stage next. Each warpgroup has an x stage of its own (and two store
 //   barriers), so that every barrier's phases are waited for in order by the
 //   one warpgroup that uses it: with one ring shared by both, a warpgroup
 //   could wait on a stage's next phase before the other one's had completed,
@@ -62,10 +62,11 @@ constexpr int kHalf = 128 * 128;        // one 64-column half of a 128-row tile
 constexpr int kTile = 2 * kHalf;        // a 128-row tile of q or x
 template <int NF>  // camera tokens rounded up to 16
 struct CamLayout {
-  // x stages per epilogue warpgroup (2 where shared memory allows), q stages
-  static constexpr int kXPerWg = NF <= 32 ? 2 : 1;
+  // x stages per epilogue warpgroup, q stages (measured: 3 q stages and one x
+  // stage per warpgroup beat 2 and 2)
+  static constexpr int kXPerWg = 1;
   static constexpr int kXStages = 2 * kXPerWg;
-  static constexpr int kQStages = NF <= 32 ? 2 : 3;
+  static constexpr int kQStages = 3;
   static constexpr int kKVHalf = NF * 128;           // a 64-column half of K or V
   static constexpr int kKV = 4 * kKVHalf;            // K and V of one head
   // barriers (8 bytes each) and control words in the first 1024 bytes
